@@ -1,0 +1,384 @@
+"""Pins of the float64 oracle against what the VideoMLA pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: figures printed on the pages
+(tests/golden/paper_figures.json), closed forms, the textbook complex-number form of 1-D RoPE,
+brute-force scalar loops on tiny inputs, an operational simulation of the streaming window, and
+torch's float64 scaled_dot_product_attention for the MLA == MHA identity.
+"""
+import itertools
+import json
+import math
+import os
+from collections import deque
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import vmla_oracle as O
+from rank_latent_kv_vmla_b200.config import TINY, WAN
+import synthetic
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "paper_figures.json")
+
+
+def _tiny_kwargs(cfg):
+    return dict(d_c=cfg.d_c, d_rope=cfg.d_rope, chunk_frames=cfg.chunk_frames, grid_h=cfg.grid_h,
+                grid_w=cfg.grid_w, pairs=(cfg.rope_pairs_t, cfg.rope_pairs_h, cfg.rope_pairs_w),
+                theta=cfg.rope_theta)
+
+
+def _f64(t):
+    return t.double().numpy()
+
+
+# ------------------------------------------------------------------------------------------------
+# Cache arithmetic printed on the pages
+# ------------------------------------------------------------------------------------------------
+def test_cache_arithmetic_matches_printed_figures():
+    g = json.load(open(GOLDEN))
+    n_h, d_h, d_c, d_r = g["n_heads"]["value"], g["d_h"]["value"], g["d_c"]["value"], g["d_rope"]["value"]
+    assert n_h * d_h == g["per_head_k_scalars_all_heads"]["value"]
+    assert O.dense_scalars_per_token(n_h, d_h) == 3072
+    assert O.latent_scalars_per_token(d_c, d_r) == 224
+    red = 100.0 * O.memory_reduction(n_h, d_h, d_c, d_r)
+    assert round(red, g["reduction_percent"]["decimals"]) == g["reduction_percent"]["value"]
+    # ~6.0 GB dense cache for 21 latent frames of Wan-1.3B under the stated reading
+    tokens = 21 * 30 * 52
+    gb = 30 * tokens * O.dense_scalars_per_token(n_h, d_h) * 2 / 1e9
+    assert round(gb, 1) == g["dense_cache_gb_21_frames"]["value"]
+    # the config presets carry the same figures
+    assert WAN.dense_scalars_per_token() == 3072 and WAN.latent_scalars_per_token() == 224
+
+
+def test_memory_reduction_changes_with_each_term():
+    base = O.memory_reduction(12, 128, 192, 32)
+    assert O.memory_reduction(12, 128, 128, 32) > base      # smaller latent -> larger saving
+    assert O.memory_reduction(12, 128, 192, 64) < base      # larger rope key -> smaller saving
+    assert O.memory_reduction(24, 128, 192, 32) > base      # more heads in the dense layout
+    assert O.memory_reduction(12, 64, 192, 32) < base       # narrower heads
+
+
+# ------------------------------------------------------------------------------------------------
+# Positions
+# ------------------------------------------------------------------------------------------------
+def test_token_positions_raster_enumeration():
+    gh, gw, f0, nframes = 3, 5, 7, 2
+    expect = [(f, i, j) for f in range(f0, f0 + nframes) for i in range(gh) for j in range(gw)]
+    got = O.token_positions(f0, nframes * gh * gw, gh, gw)
+    assert [tuple(r) for r in got.tolist()] == expect
+
+
+# ------------------------------------------------------------------------------------------------
+# 3D-RoPE
+# ------------------------------------------------------------------------------------------------
+def test_rope_hand_values():
+    # pairs (2, 1, 1), theta = 1e4: frame pairs turn at 1 and 1e4^(-1/2) = 0.01; row and column at 1
+    u = np.array([1.0, 0.0] * 4)
+    out = O.rope3d(u, np.array([3, 2, 1]), (2, 1, 1), 1e4)
+    expect = [math.cos(3), math.sin(3), math.cos(0.03), math.sin(0.03),
+              math.cos(2), math.sin(2), math.cos(1), math.sin(1)]
+    np.testing.assert_allclose(out, expect, rtol=0, atol=1e-15)
+    # the second component of a pair turns the same way: (0, 1) -> (-sin, cos)
+    out2 = O.rope3d(np.array([0.0, 1.0] * 4), np.array([3, 2, 1]), (2, 1, 1), 1e4)
+    np.testing.assert_allclose(out2[0:2], [-math.sin(3), math.cos(3)], atol=1e-15)
+
+
+def test_rope_single_axis_is_textbook_1d_rope():
+    """With all pairs on the frame axis, 3D-RoPE is 1-D RoPE: pair m is the complex number
+    u[2m] + i u[2m+1] multiplied by exp(i * pos * theta^(-2m/d))."""
+    rng = np.random.default_rng(0)
+    d = 16
+    u = rng.standard_normal((5, d))
+    pos = np.array([[0, 0, 0], [1, 0, 0], [7, 0, 0], [100, 0, 0], [12345, 0, 0]])
+    got = O.rope3d(u, pos, (d // 2, 0, 0), 10000.0)
+    z = u[:, 0::2] + 1j * u[:, 1::2]
+    m = np.arange(d // 2)
+    zr = z * np.exp(1j * pos[:, :1] * 10000.0 ** (-2.0 * m / d))
+    np.testing.assert_allclose(got[:, 0::2], zr.real, atol=1e-12)
+    np.testing.assert_allclose(got[:, 1::2], zr.imag, atol=1e-12)
+
+
+def test_rope_zero_position_identity_and_norm():
+    rng = np.random.default_rng(1)
+    u = rng.standard_normal((50, 32))
+    pairs = (6, 5, 5)
+    np.testing.assert_array_equal(O.rope3d(u, np.zeros(3, dtype=np.int64), pairs, 1e4), u)
+    pos = rng.integers(0, 300, size=(50, 3))
+    r = O.rope3d(u, pos, pairs, 1e4)
+    # each pair keeps its length (a rotation), hence the vector keeps its norm
+    np.testing.assert_allclose(np.hypot(r[:, 0::2], r[:, 1::2]), np.hypot(u[:, 0::2], u[:, 1::2]),
+                               rtol=1e-13)
+
+
+def test_rope_relative_position_invariance():
+    """q(p) . k(p') depends only on p - p': shifting both positions by any (df, di, dj) leaves it."""
+    rng = np.random.default_rng(2)
+    pairs = (6, 5, 5)
+    q = rng.standard_normal((200, 32))
+    k = rng.standard_normal((200, 32))
+    pq = rng.integers(0, 60, size=(200, 3))
+    pk = rng.integers(0, 60, size=(200, 3))
+    s0 = np.sum(O.rope3d(q, pq, pairs, 1e4) * O.rope3d(k, pk, pairs, 1e4), axis=-1)
+    for shift in ([5, 0, 0], [0, 3, 0], [0, 0, 11], [17, -4, 9]):
+        sh = np.array(shift)
+        s1 = np.sum(O.rope3d(q, pq + sh, pairs, 1e4) * O.rope3d(k, pk + sh, pairs, 1e4), axis=-1)
+        np.testing.assert_allclose(s1, s0, rtol=1e-10, atol=1e-10)
+    # and it is not invariant to a shift of only one side (so the test can fail)
+    s2 = np.sum(O.rope3d(q, pq + np.array([1, 1, 1]), pairs, 1e4) * O.rope3d(k, pk, pairs, 1e4), axis=-1)
+    assert np.max(np.abs(s2 - s0)) > 1e-2
+
+
+def test_rope_axis_blocks_follow_t_h_w_order():
+    """Moving only the row index turns only the P_h row pairs (pairs P_t .. P_t+P_h-1)."""
+    u = np.ones(32)
+    pairs = (6, 5, 5)
+    base = O.rope3d(u, np.array([4, 2, 9]), pairs, 1e4)
+    moved = O.rope3d(u, np.array([4, 3, 9]), pairs, 1e4)
+    changed = np.nonzero(np.abs(moved - base) > 1e-14)[0] // 2
+    assert set(changed.tolist()) == set(range(6, 11))
+
+
+# ------------------------------------------------------------------------------------------------
+# Compression, cache and sliding window (brute force)
+# ------------------------------------------------------------------------------------------------
+def test_compress_against_scalar_loops():
+    cfg = TINY
+    inp = synthetic.draw_layer(cfg, batch=1, seed=11, n_chunks=1)
+    x = _f64(inp.x_chunks[0][0])
+    w = _f64(inp.w_dkv_kr)
+    pos = O.token_positions(5, x.shape[0], cfg.grid_h, cfg.grid_w)
+    pairs = (cfg.rope_pairs_t, cfg.rope_pairs_h, cfg.rope_pairs_w)
+    c, k_r = O.compress(x, w, cfg.d_c, pos, pairs, cfg.rope_theta)
+    for t in range(x.shape[0]):
+        for r in range(cfg.d_c):
+            ref = sum(w[r, d] * x[t, d] for d in range(cfg.dim))
+            assert abs(c[t, r] - ref) < 1e-12
+        raw = [sum(w[cfg.d_c + r, d] * x[t, d] for d in range(cfg.dim)) for r in range(cfg.d_rope)]
+        f, i, j = pos[t]
+        axis_pos = [f] * cfg.rope_pairs_t + [i] * cfg.rope_pairs_h + [j] * cfg.rope_pairs_w
+        local = list(range(cfg.rope_pairs_t)) + list(range(cfg.rope_pairs_h)) + list(range(cfg.rope_pairs_w))
+        size = [cfg.rope_pairs_t] * cfg.rope_pairs_t + [cfg.rope_pairs_h] * cfg.rope_pairs_h + \
+               [cfg.rope_pairs_w] * cfg.rope_pairs_w
+        for p in range(cfg.d_rope // 2):
+            ang = axis_pos[p] * cfg.rope_theta ** (-local[p] / size[p])
+            a, b = raw[2 * p], raw[2 * p + 1]
+            assert abs(k_r[t, 2 * p] - (a * math.cos(ang) - b * math.sin(ang))) < 1e-12
+            assert abs(k_r[t, 2 * p + 1] - (a * math.sin(ang) + b * math.cos(ang))) < 1e-12
+
+
+def test_ring_matches_explicit_ring_writes():
+    """Append 6 one-frame chunks into a 3-frame window: the expected ring equals an explicit ring that
+    writes frame f into slot f mod W (evicting f - W), checked after every append."""
+    W, T, d = 3, 4, 2
+    hist = np.arange(6 * T * d, dtype=np.float64).reshape(6 * T, d)
+    ring = np.full((W * T, d), np.nan)
+    for fw in range(1, 7):
+        f = fw - 1
+        s = f % W
+        ring[s * T:(s + 1) * T] = hist[f * T:(f + 1) * T]
+        plane, written = O.ring_from_history(hist[:fw * T], fw, W, T)
+        np.testing.assert_array_equal(np.isnan(plane[:, 0]), np.isnan(ring[:, 0]))
+        np.testing.assert_array_equal(plane[written], ring[written])
+        assert written.sum() == min(fw, W) * T
+    assert [O.frame_of_slot(s, 6, W) for s in range(W)] == [3, 4, 5]
+    assert [O.frame_of_slot(s, 2, W) for s in range(W)] == [0, 1, -1]
+    assert O.frame_of_slot(0, 0, W) == -1
+
+
+def test_window_mask_matches_streaming_simulation():
+    """The block-causal + window mask equals what a streaming generator sees: chunk k attends, right
+    after appending its own frames, to exactly the frames held in a W-frame sliding window."""
+    F, T = 2, 3
+    for W in (2, 3, 4, 5, 8, 20):
+        n_chunks = 5
+        key_frames = np.repeat(np.arange(n_chunks * F), T)
+        hi = O.query_chunk_end(0, n_chunks * F * T, F, T)
+        mask = O.visible(hi, key_frames, W)
+        window = deque(maxlen=W)
+        for k in range(n_chunks):
+            for f in range(k * F, (k + 1) * F):
+                window.append(f)
+            allowed = set(window)
+            rows = range(k * F * T, (k + 1) * F * T)
+            for n in rows:
+                got = {int(key_frames[t]) for t in np.nonzero(mask[n])[0]}
+                assert got == allowed, (W, k, n)
+
+
+# ------------------------------------------------------------------------------------------------
+# Attention: brute force, special cases, absorbed == reconstructed, MLA == MHA (library routine)
+# ------------------------------------------------------------------------------------------------
+def _tiny_history(cfg, seed, n_chunks, q_gain=1.0):
+    inp = synthetic.draw_layer(cfg, batch=1, seed=seed, n_chunks=n_chunks, q_gain=q_gain)
+    hist = O.build_history(inp.x_chunks, _f64(inp.w_dkv_kr), 0, **_tiny_kwargs(cfg))
+    return inp, hist
+
+
+def _ref(cfg, inp, hist, first_frame, rows=None, q_nope=None, q_rope=None):
+    qn = _f64(inp.q_nope[0]) if q_nope is None else q_nope
+    qr = _f64(inp.q_rope[0]) if q_rope is None else q_rope
+    rows = np.arange(qn.shape[0]) if rows is None else rows
+    return O.layer_reference(hist, qn, qr, _f64(inp.w_uk), _f64(inp.w_uv), first_frame=first_frame,
+                             query_rows=rows, chunk_frames=cfg.chunk_frames,
+                             window_frames=cfg.window_frames, grid_h=cfg.grid_h, grid_w=cfg.grid_w,
+                             pairs=(cfg.rope_pairs_t, cfg.rope_pairs_h, cfg.rope_pairs_w),
+                             theta=cfg.rope_theta, scale=cfg.scale)
+
+
+def test_attention_against_scalar_loops():
+    cfg = TINY
+    n_chunks = 5                     # frames 0..4, window 3: frames 0, 1 evicted
+    inp, hist = _tiny_history(cfg, 21, n_chunks)
+    f0 = (n_chunks - 1) * cfg.chunk_frames
+    ref = _ref(cfg, inp, hist, f0)
+    qn, qr = _f64(inp.q_nope[0]), _f64(inp.q_rope[0])
+    wuk, wuv = _f64(inp.w_uk), _f64(inp.w_uv)
+    T = cfg.tokens_per_frame
+    for n in range(qn.shape[0]):
+        f, i, j = f0 + n // T, (n % T) // cfg.grid_w, n % cfg.grid_w
+        for h in range(cfg.n_heads):
+            # rotate the query by explicit pair loops
+            qrot = []
+            for p in range(cfg.d_rope // 2):
+                if p < cfg.rope_pairs_t:
+                    ang = f * cfg.rope_theta ** (-p / cfg.rope_pairs_t)
+                elif p < cfg.rope_pairs_t + cfg.rope_pairs_h:
+                    ang = i * cfg.rope_theta ** (-(p - cfg.rope_pairs_t) / cfg.rope_pairs_h)
+                else:
+                    ang = j * cfg.rope_theta ** (-(p - cfg.rope_pairs_t - cfg.rope_pairs_h) / cfg.rope_pairs_w)
+                a, b = qr[n, h, 2 * p], qr[n, h, 2 * p + 1]
+                qrot += [a * math.cos(ang) - b * math.sin(ang), a * math.sin(ang) + b * math.cos(ang)]
+            scores, vals = [], []
+            for t in range(hist.c.shape[0]):
+                kf = hist.frames[t]
+                if not (f0 + cfg.chunk_frames - cfg.window_frames <= kf < f0 + cfg.chunk_frames):
+                    continue
+                knope = [sum(wuk[h, r, m] * hist.c[t, m] for m in range(cfg.d_c)) for r in range(cfg.d_nope)]
+                s = sum(qn[n, h, r] * knope[r] for r in range(cfg.d_nope))
+                s += sum(qrot[r] * hist.k_r[t, r] for r in range(cfg.d_rope))
+                scores.append(s * cfg.scale)
+                vals.append([sum(wuv[h, r, m] * hist.c[t, m] for m in range(cfg.d_c)) for r in range(cfg.d_v)])
+            mx = max(scores)
+            e = [math.exp(s - mx) for s in scores]
+            z = sum(e)
+            o = [sum(e[t] * vals[t][r] for t in range(len(e))) / z for r in range(cfg.d_v)]
+            np.testing.assert_allclose(ref["o"][n, h], o, rtol=1e-11, atol=1e-12)
+            assert abs(ref["lse"][n, h] - (math.log(z) + mx)) < 1e-11
+        assert len(scores) == cfg.window_frames * T
+
+
+def test_softmax_rows_sum_to_one_and_lse():
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((7, 3, 8))
+    k = rng.standard_normal((20, 3, 8))
+    v = rng.standard_normal((20, 3, 4))
+    mask = rng.random((7, 20)) < 0.6
+    mask[:, 0] = True
+    o, lse, p = O.mha(q, k, v, mask, 0.3)
+    np.testing.assert_allclose(p.sum(-1), 1.0, rtol=1e-14)
+    assert np.all(p[np.broadcast_to(~mask[:, None, :], p.shape)] == 0)
+    s = np.einsum('nhd,thd->nht', q, k) * 0.3
+    np.testing.assert_allclose(lse, np.log(np.sum(np.where(mask[:, None, :], np.exp(s), 0), -1)), rtol=1e-13)
+
+
+def test_single_visible_key_returns_its_value():
+    rng = np.random.default_rng(6)
+    q = rng.standard_normal((4, 2, 8)) * 30.0
+    k = rng.standard_normal((9, 2, 8))
+    v = rng.standard_normal((9, 2, 5))
+    mask = np.zeros((4, 9), dtype=bool)
+    mask[np.arange(4), [0, 3, 8, 5]] = True
+    o, _, _ = O.mha(q, k, v, mask, 1.0)
+    np.testing.assert_allclose(o, v[[0, 3, 8, 5]], rtol=1e-14)
+
+
+def test_zero_query_gives_mean_of_visible_values():
+    cfg = TINY
+    inp, hist = _tiny_history(cfg, 31, 4)
+    f0 = 3 * cfg.chunk_frames
+    qn = np.zeros_like(_f64(inp.q_nope[0]))
+    qr = np.zeros_like(_f64(inp.q_rope[0]))
+    ref = _ref(cfg, inp, hist, f0, q_nope=qn, q_rope=qr)
+    vis = (hist.frames >= f0 + 1 - cfg.window_frames) & (hist.frames < f0 + 1)
+    v = np.einsum('hvc,tc->thv', _f64(inp.w_uv), hist.c[vis])
+    np.testing.assert_allclose(ref["o"], np.broadcast_to(v.mean(0), ref["o"].shape), rtol=1e-12)
+    np.testing.assert_allclose(ref["o_latent"], np.broadcast_to(hist.c[vis].mean(0), ref["o_latent"].shape),
+                               rtol=1e-12)
+
+
+@pytest.mark.parametrize("q_gain", [1.0, 8.0])
+def test_absorbed_equals_reconstructed(q_gain):
+    cfg = TINY
+    inp, hist = _tiny_history(cfg, 41, 4, q_gain=q_gain)
+    f0 = 3 * cfg.chunk_frames
+    ref = _ref(cfg, inp, hist, f0)
+    o_lat, lse = O.latent_attention(ref["q_abs"], hist.c, hist.k_r, ref["mask"], cfg.scale)
+    np.testing.assert_allclose(o_lat, ref["o_latent"], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, ref["lse"], rtol=1e-12)
+    np.testing.assert_allclose(O.value_up(o_lat, _f64(inp.w_uv)), ref["o"], rtol=1e-11, atol=1e-13)
+
+
+def test_mla_equals_textbook_mha_via_torch_sdpa():
+    """With dense per-head weights built as W_K,h = [W^K_up,h W^KV_down ; W^KR] (rope rows rotated)
+    and W_V,h = W^V_up,h W^KV_down, the MLA layer is ordinary MHA: compare against torch's float64
+    scaled_dot_product_attention (default scale 1/sqrt(d_h)) with an explicit boolean mask."""
+    cfg = TINY.replace(window_frames=2, chunk_frames=1)
+    n_chunks = 4
+    inp, hist = _tiny_history(cfg, 51, n_chunks)
+    f0 = (n_chunks - 1) * cfg.chunk_frames
+    ref = _ref(cfg, inp, hist, f0)
+
+    w = torch.from_numpy(_f64(inp.w_dkv_kr))
+    w_dkv, w_kr = w[:cfg.d_c], w[cfg.d_c:]
+    wuk, wuv = torch.from_numpy(_f64(inp.w_uk)), torch.from_numpy(_f64(inp.w_uv))
+    xs = torch.cat([torch.from_numpy(_f64(x[0])) for x in inp.x_chunks])          # [T_all, D]
+    pairs = (cfg.rope_pairs_t, cfg.rope_pairs_h, cfg.rope_pairs_w)
+    pos_k = np.concatenate([O.token_positions(k * cfg.chunk_frames, cfg.chunk_tokens, cfg.grid_h, cfg.grid_w)
+                            for k in range(n_chunks)])
+    k_heads, v_heads = [], []
+    for h in range(cfg.n_heads):
+        wk_h = wuk[h] @ w_dkv                                                       # [d_nope, D]
+        k_nope = xs @ wk_h.T
+        k_rope = torch.from_numpy(O.rope3d((xs @ w_kr.T).numpy(), pos_k, pairs, cfg.rope_theta))
+        k_heads.append(torch.cat([k_nope, k_rope], -1))
+        v_heads.append(xs @ (wuv[h] @ w_dkv).T)
+    K = torch.stack(k_heads, 0)                                                     # [H, T, d_h]
+    V = torch.stack(v_heads, 0)
+    pos_q = O.token_positions(f0, cfg.chunk_tokens, cfg.grid_h, cfg.grid_w)
+    q_rot = O.rotate_query(_f64(inp.q_rope[0]), pos_q, pairs, cfg.rope_theta)
+    Q = torch.cat([torch.from_numpy(_f64(inp.q_nope[0])), torch.from_numpy(q_rot)], -1).transpose(0, 1)
+    key_frames = torch.from_numpy(pos_k[:, 0])
+    allowed = (key_frames >= f0 + cfg.chunk_frames - cfg.window_frames) & (key_frames < f0 + cfg.chunk_frames)
+    attn_mask = allowed[None, None, :].expand(cfg.n_heads, cfg.chunk_tokens, -1)
+    o = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=attn_mask)
+    np.testing.assert_allclose(ref["o"], o.transpose(0, 1).numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_streaming_calls_equal_one_block_causal_call():
+    """With a window that holds every frame, one call over 4 chunks (block-causal) equals 4 streaming
+    calls, each made right after appending its own chunk."""
+    cfg = TINY.replace(window_frames=8)
+    n_chunks = 4
+    inp = synthetic.draw_layer(cfg, batch=1, seed=61, n_chunks=n_chunks, n_query_chunks=n_chunks)
+    hist = O.build_history(inp.x_chunks, _f64(inp.w_dkv_kr), 0, **_tiny_kwargs(cfg))
+    qn, qr = _f64(inp.q_nope[0]), _f64(inp.q_rope[0])
+    whole = _ref(cfg, inp, hist, 0, q_nope=qn, q_rope=qr)
+    per = cfg.chunk_tokens
+    for k in range(n_chunks):
+        part = O.build_history(inp.x_chunks[:k + 1], _f64(inp.w_dkv_kr), 0, **_tiny_kwargs(cfg))
+        one = _ref(cfg, inp, part, k * cfg.chunk_frames, q_nope=qn[k * per:(k + 1) * per],
+                   q_rope=qr[k * per:(k + 1) * per])
+        np.testing.assert_allclose(whole["o"][k * per:(k + 1) * per], one["o"], rtol=1e-12, atol=1e-14)
+    # chunk 0 sees only itself; the last chunk sees everything
+    assert whole["mask"][0].sum() == per and whole["mask"][-1].sum() == n_chunks * per
+
+
+def test_layer_reference_row_sampling_is_consistent():
+    cfg = TINY
+    inp, hist = _tiny_history(cfg, 71, 3)
+    full = _ref(cfg, inp, hist, 2)
+    rows = np.array([0, 5, 15])
+    part = _ref(cfg, inp, hist, 2, rows=rows)
+    for key in ("o", "o_latent", "lse", "q_abs"):
+        np.testing.assert_array_equal(part[key], full[key][rows])
