@@ -1,0 +1,462 @@
+"""Benchmark of the VideoMLA latent-attention layer step on B200.
+
+One step = one streaming chunk of one Wan-1.3B-shaped layer through the whole path:
+compress + 3D-RoPE + ring append (4680 tokens), absorbed query, latent attention of 4680 x 12 query
+rows against the full 21-frame window (32760 cached tokens), and the value up-projection.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B] [--impl reference]
+
+Prints one JSON line (rank 0).  ``value`` is latent-attention TFLOP/s (2*B*H*Nq*Nk*(2*d_c + d_rope)
+algorithmic flops per step, whole step timed on the device with CUDA events, L2 flushed between
+steps), summed over ranks (each rank runs its own batch: weak scaling).  ``--impl reference`` times
+the float64 CPU oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+
+from rank_latent_kv_vmla_b200.config import WAN
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+N_INPUT_SETS = 4          # distinct x / q sets cycled through the steps (all resident in HBM)
+FLUSH_BYTES = 512 << 20   # > 126 MB L2
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--batch", type=int, default=1, help="sequences per GPU")
+    ap.add_argument("--impl", default="vmla", choices=["vmla", "reference"])
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense MHA comparison arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------------------------
+# Workload arithmetic
+# ------------------------------------------------------------------------------------------------
+def attention_flops(cfg, batch) -> float:
+    """Algorithmic flops of one latent-attention call: 2*B*H*Nq*Nk*(2*d_c + d_rope)."""
+    return 2.0 * batch * cfg.n_heads * cfg.chunk_tokens * cfg.window_tokens * (2 * cfg.d_c + cfg.d_rope)
+
+
+def dense_attention_flops(cfg, batch) -> float:
+    return 2.0 * batch * cfg.n_heads * cfg.chunk_tokens * cfg.window_tokens * (cfg.d_h + cfg.d_v)
+
+
+def kernel_bytes(cfg, batch):
+    """Algorithmic HBM bytes per launch of the HBM-bound steps (bf16)."""
+    e = 2
+    nq, H = cfg.chunk_tokens, cfg.n_heads
+    return {
+        "compress_append": batch * nq * (cfg.dim + cfg.d_c + cfg.d_rope) * e + (cfg.d_c + cfg.d_rope) * cfg.dim * e,
+        "absorb_q": batch * nq * H * (cfg.d_nope + cfg.d_rope + cfg.d_qk) * e + H * cfg.d_nope * cfg.d_c * e,
+        "value_up": batch * nq * H * (cfg.d_c + cfg.d_v) * e + H * cfg.d_v * cfg.d_c * e,
+    }
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def traffic_for(kernel: str, source_hash: str):
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        ent = t.get(kernel)
+        if ent and ent.get("source_hash") == source_hash:
+            return ent.get("bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+def source_hash(names):
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        p = os.path.join(ROOT, "rank_latent_kv_vmla_b200", "csrc", n)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# Distributed plumbing (one process per GPU; timing collective only)
+# ------------------------------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        rank = int(os.environ["RANK"])
+        local = int(os.environ.get("LOCAL_RANK", rank))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        return rank, world, local
+    return 0, 1, 0
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and --impl reference)
+# ------------------------------------------------------------------------------------------------
+def oracle_sample(cfg, batch, seed, n_rows):
+    """Time the oracle's layer step on a bounded sample: compress the new chunk, then the
+    non-absorbed attention of ``n_rows`` query tokens (all heads) over the full window."""
+    from oracle import vmla_oracle as O
+    import synthetic
+    inp = synthetic.draw_layer(cfg, batch=1, seed=seed, n_chunks=cfg.window_frames // cfg.chunk_frames)
+    xs = [x.double().numpy() for x in inp.x_chunks]
+    w = inp.w_dkv_kr.double().numpy()
+    kw = dict(d_c=cfg.d_c, d_rope=cfg.d_rope, chunk_frames=cfg.chunk_frames, grid_h=cfg.grid_h,
+              grid_w=cfg.grid_w, pairs=(cfg.rope_pairs_t, cfg.rope_pairs_h, cfg.rope_pairs_w),
+              theta=cfg.rope_theta)
+    hist = O.build_history(xs[:-1], w, 0, **kw)
+    f0 = (len(xs) - 1) * cfg.chunk_frames
+    qn, qr = inp.q_nope[0].double().numpy(), inp.q_rope[0].double().numpy()
+    rows = np.linspace(0, cfg.chunk_tokens - 1, n_rows).astype(np.int64)
+    t0 = time.perf_counter()
+    pos = O.token_positions(f0, cfg.chunk_tokens, cfg.grid_h, cfg.grid_w)
+    c, k_r = O.compress(xs[-1][0], w, cfg.d_c, pos, kw["pairs"], cfg.rope_theta)
+    hist.append(c, k_r, pos[:, 0])
+    O.layer_reference(hist, qn, qr, inp.w_uk.double().numpy(), inp.w_uv.double().numpy(),
+                      first_frame=f0, query_rows=rows, chunk_frames=cfg.chunk_frames,
+                      window_frames=cfg.window_frames, grid_h=cfg.grid_h, grid_w=cfg.grid_w,
+                      pairs=kw["pairs"], theta=cfg.rope_theta, scale=cfg.scale)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(cfg, target_s):
+    cores = len(os.sched_getaffinity(0))
+    probe = 32
+    t_probe = oracle_sample(cfg, 1, 4321, probe)
+    n_rows = int(min(cfg.chunk_tokens, max(probe, probe * target_s / max(t_probe, 1e-3))))
+    t = oracle_sample(cfg, 1, 4321, n_rows)
+    flops = attention_flops(cfg, 1) * n_rows / cfg.chunk_tokens
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "query_tokens_per_s": n_rows / t,
+            "sample": f"float64 NumPy oracle, one layer step of the Wan-1.3B layer restricted to {n_rows} "
+                      f"of {cfg.chunk_tokens} query tokens (all {cfg.n_heads} heads, full 21-frame window, "
+                      f"non-absorbed K/V materialised), {t:.1f} s; value = those rows' latent-attention flops / time"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = WAN
+    cores = len(os.sched_getaffinity(0))
+    n_rows = 48
+    for _ in range(args.warmup):
+        oracle_sample(cfg, 1, 4321, n_rows)
+    times = [oracle_sample(cfg, 1, 4321, n_rows) for _ in range(args.steps)]
+    t = sum(times)
+    flops = attention_flops(cfg, 1) * n_rows / cfg.chunk_tokens * args.steps
+    val = flops / t / 1e12
+    line = {"metric": "latent-attention TFLOP/s (Wan-1.3B layer step, B200 BF16 TC peak fraction)",
+            "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "wan1.3b_layer_stream_step", "batch_per_gpu": 1,
+                       "query_tokens": cfg.chunk_tokens, "cached_tokens": cfg.window_tokens},
+            "impl": "reference",
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{n_rows} of {cfg.chunk_tokens} query tokens per step (all heads), "
+                                       "float64 NumPy oracle incl. the chunk's compression"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from rank_latent_kv_vmla_b200 import vmla as V
+    import synthetic
+
+    cfg = WAN
+    B = args.batch
+    pk, pk_src = peaks()
+    seed = 1234 + 1 + 1000 * rank
+    prefill = cfg.window_frames // cfg.chunk_frames - 1          # 6 chunks: frames 0..17
+    inp = synthetic.draw_layer(cfg, batch=B, seed=seed, n_chunks=prefill + N_INPUT_SETS)
+    extra_q = [synthetic.draw_queries(cfg, B, seed + 7 + i) for i in range(N_INPUT_SETS)]
+    w = inp.w_dkv_kr.to(dev)
+    w_uk, w_uv = inp.w_uk.to(dev), inp.w_uv.to(dev)
+    xs = [x.to(dev) for x in inp.x_chunks[prefill:]]
+    qs = [(qn.to(dev), qr.to(dev)) for qn, qr in extra_q]
+    cache = V.LatentCache(cfg, B, device=dev)
+    for x in inp.x_chunks[:prefill]:
+        V.compress_append(cfg, x.to(dev), w, cache)
+    bufs = {"q_abs": torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_qk), dtype=torch.bfloat16, device=dev),
+            "o_latent": torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_c), dtype=torch.bfloat16, device=dev),
+            "o": torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    names = ["compress_append", "absorb_q", "latent_attention", "value_up"]
+
+    def step(i, ev=None):
+        x = xs[i % N_INPUT_SETS]
+        qn, qr = qs[i % N_INPUT_SETS]
+        f0 = cache.frames_written
+        if ev: ev[0].record(stream)
+        V.compress_append(cfg, x, w, cache, f0)
+        if ev: ev[1].record(stream)
+        V.absorb_q(cfg, qn, qr, w_uk, f0, out=bufs["q_abs"])
+        if ev: ev[2].record(stream)
+        V.latent_attention(cfg, bufs["q_abs"], cache, f0, out=bufs["o_latent"])
+        if ev: ev[3].record(stream)
+        V.value_up(cfg, bufs["o_latent"], w_uv, out=bufs["o"])
+        if ev: ev[4].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+        flush.zero_()
+    torch.cuda.synchronize()
+    assert V.device_status() == 0
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    launches0 = V.launch_count()
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i, evs[i])
+        flush.zero_()
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    launches = V.launch_count() - launches0
+    clk = clocks.stop()
+    barrier(world)
+    per_kernel = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)] for j, n in enumerate(names)}
+    step_ms = [evs[i][0].elapsed_time(evs[i][4]) for i in range(args.steps)]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    assert V.device_status() == 0
+
+    f_step = attention_flops(cfg, B)
+    value = world * f_step * args.steps / (total_ms * 1e-3) / 1e12
+    q_tok_s = world * B * cfg.chunk_tokens * args.steps / (total_ms * 1e-3)
+    k3_ms = statistics.mean(per_kernel["latent_attention"])
+    k3_tflops = f_step / (k3_ms * 1e-3) / 1e12
+    kb = kernel_bytes(cfg, B)
+    kernels = {"latent_attention": {"ms": k3_ms, "tflops": k3_tflops}}
+    for n in ("compress_append", "absorb_q", "value_up"):
+        ms = statistics.mean(per_kernel[n])
+        kernels[n] = {"ms": ms, "gbs": kb[n] / (ms * 1e-3) / 1e9, "frac_hbm": kb[n] / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
+    k3_src = source_hash(["tc_attention.cu", "tc_kernels.cuh", "ptx_sm100.cuh"])
+    roofline = {"bound": "tensor", "kernel": "latent_attention", "achieved": k3_tflops,
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": k3_tflops / pk["bf16_tflops"],
+                "peak_source": f"{pk_src} bf16 burst (MEASURED_PEAKS.json)" if pk_src == "measured" else "fallback 1.59 PFLOP/s",
+                "frac_of_sustained": k3_tflops / pk["bf16_tflops_sustained"],
+                "flops_per_launch": f_step,
+                "traffic": traffic_for("latent_attention_wan_b%d" % B, k3_src)}
+
+    # ---- end to end through the public API with host buffers (pinned) ----
+    hx = [x.cpu().pin_memory() for x in xs]
+    hq = [(qn.cpu().pin_memory(), qr.cpu().pin_memory()) for qn, qr in qs]
+    ho = torch.empty(bufs["o"].shape, dtype=torch.bfloat16).pin_memory()
+    dx = torch.empty_like(xs[0]); dqn = torch.empty_like(qs[0][0]); dqr = torch.empty_like(qs[0][1])
+    h2d = dx.numel() * 2 + dqn.numel() * 2 + dqr.numel() * 2
+    d2h = ho.numel() * 2
+
+    def e2e_step(i):
+        dx.copy_(hx[i % N_INPUT_SETS], non_blocking=True)
+        dqn.copy_(hq[i % N_INPUT_SETS][0], non_blocking=True)
+        dqr.copy_(hq[i % N_INPUT_SETS][1], non_blocking=True)
+        f0 = cache.frames_written
+        V.compress_append(cfg, dx, w, cache, f0)
+        V.absorb_q(cfg, dqn, dqr, w_uk, f0, out=bufs["q_abs"])
+        V.latent_attention(cfg, bufs["q_abs"], cache, f0, out=bufs["o_latent"])
+        V.value_up(cfg, bufs["o_latent"], w_uv, out=bufs["o"])
+        ho.copy_(bufs["o"], non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i)
+    e2e_steps = max(10, args.steps // 4)
+    torch.cuda.synchronize()
+    barrier(world)
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    for i in range(e2e_steps):
+        flush.zero_()
+        ea.record(stream)
+        e2e_step(i)
+        eb.record(stream)
+        eb.synchronize()
+        e2e_ms += ea.elapsed_time(eb)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e = {"value": world * f_step * e2e_steps / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": e2e_ms / e2e_steps}
+
+    # ---- dense per-head MHA comparison on the same shapes (not part of `value`) ----
+    comparison = None
+    if not args.no_dense:
+        w_kv = synthetic.draw_dense_weights(cfg, seed + 3).to(dev)
+        dcache = V.DenseCache(cfg, B, device=dev)
+        for x in inp.x_chunks[:prefill]:
+            V.dense_append(cfg, x.to(dev), w_kv, dcache)
+        dq = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_h), dtype=torch.bfloat16, device=dev)
+        do = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
+        dsteps = max(10, args.steps // 4)
+        devs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(dsteps)]
+
+        def dstep(i, ev):
+            f0 = dcache.frames_written
+            ev[0].record(stream)
+            V.dense_append(cfg, xs[i % N_INPUT_SETS], w_kv, dcache, f0)
+            ev[1].record(stream)
+            V.rope_q(cfg, qs[i % N_INPUT_SETS][0], qs[i % N_INPUT_SETS][1], f0, out=dq)
+            ev[2].record(stream)
+            V.dense_mha(cfg, dq, dcache, f0, out=do)
+            ev[3].record(stream)
+
+        for i in range(3):
+            dstep(i, devs[0])
+            flush.zero_()
+        for i in range(dsteps):
+            dstep(i, devs[i])
+            flush.zero_()
+        torch.cuda.synchronize()
+        d_step_ms = statistics.mean(devs[i][0].elapsed_time(devs[i][3]) for i in range(dsteps))
+        d_mha_ms = statistics.mean(devs[i][2].elapsed_time(devs[i][3]) for i in range(dsteps))
+        comparison = {"dense_step_ms": d_step_ms, "dense_mha_ms": d_mha_ms,
+                      "dense_mha_tflops": dense_attention_flops(cfg, B) / (d_mha_ms * 1e-3) / 1e12,
+                      "latent_step_ms": statistics.mean(step_ms), "latent_attention_ms": k3_ms,
+                      "step_speedup_vs_dense": d_step_ms / statistics.mean(step_ms),
+                      "attention_speedup_vs_dense": d_mha_ms / k3_ms,
+                      "cache_bytes_latent": V.latent_cache_bytes(cfg, B),
+                      "cache_bytes_dense": V.dense_cache_bytes(cfg, B),
+                      "cache_bytes_ratio": V.latent_cache_bytes(cfg, B) / V.dense_cache_bytes(cfg, B)}
+        assert V.device_status() == 0
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(cfg, args.cpu_seconds)
+        line = {"metric": "latent-attention TFLOP/s (Wan-1.3B layer step, B200 BF16 TC peak fraction)",
+                "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "wan1.3b_layer_stream_step", "batch_per_gpu": B, "global_batch": B * world,
+                           "query_tokens": cfg.chunk_tokens, "cached_tokens": cfg.window_tokens,
+                           "heads": cfg.n_heads, "d_c": cfg.d_c, "d_rope": cfg.d_rope, "d_v": cfg.d_v,
+                           "dim": cfg.dim, "parallelism": f"dp{world} (independent sequences)",
+                           "l2": "flushed between steps (512 MB write)"},
+                "query_tokens_per_s": q_tok_s,
+                "pct_of_bf16_peak": 100.0 * value / world / pk["bf16_tflops"],
+                "roofline": roofline, "kernels": kernels, "e2e": e2e, "gpu_launches": launches,
+                "clocks": clk, "wall_s_timed": wall, "cpu_baseline": cpu, "comparison": comparison}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

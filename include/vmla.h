@@ -1,0 +1,186 @@
+/*
+ * vmla.h - C ABI of the VideoMLA latent-KV attention library (libvmla.so, sm_100a).
+ *
+ * VideoMLA ("VideoMLA: Low-Rank Latent KV Cache for Minute-Scale Autoregressive Video Diffusion",
+ * gist.science technical summary, Method items 1-4) caches, for every token t of a sliding window of
+ * latent frames, only the pair (c^KV_t, k^R_t): a content latent c^KV_t = W^KV_down x_t shared by all
+ * heads (d_c scalars) and one head-shared positional key k^R_t rotated by 3D-RoPE (d_rope scalars).
+ * Per-head content keys and values are never stored; this library never materialises them either:
+ * the key up-projection is absorbed into the query, q~_h = (W^K_up,h)^T q^nope_h, so the score of key
+ * t is  scale * (q~_h . c_t + q^R_h . k^R_t),  and the value up-projection W^V_up,h is applied once to
+ * the attention-weighted latent sum.
+ *
+ * Conventions shared by every call
+ *  - Ownership: every tensor argument is a caller-owned DEVICE buffer; the library allocates no device
+ *    memory and keeps no pointer after a call returns.  Host structs (vmla_config, vmla_cache) are
+ *    read during the call; vmla_cache.frames_written is updated by the append calls.
+ *  - Execution: work is enqueued on the caller's CUDA stream (`stream` is a cudaStream_t; NULL is the
+ *    legacy default stream) and the call returns without synchronising.
+ *  - Layout: row-major, last dimension contiguous, no padding between rows.  Every base pointer must be
+ *    16-byte aligned (VMLA_ERR_MISALIGNED otherwise).
+ *  - Element type: cfg->dtype selects VMLA_BF16 (bf16 storage, fp32 accumulation, tensor-core kernels)
+ *    or VMLA_F32 (fp32 storage and arithmetic, CUDA-core kernels).  The lse outputs are always fp32.
+ *  - Errors: arguments are validated on the host before anything is launched; on error nothing is
+ *    enqueued and a status is returned.  vmla_last_error_detail() gives a text for the calling thread.
+ *    Device-side waits are bounded: a wait that runs out sets a device status word and the kernel
+ *    returns; vmla_device_status() reads (and clears) it.
+ *
+ * Frame geometry: a latent frame is a grid_h x grid_w grid of tokens (T_f = grid_h*grid_w) in raster
+ * order; a chunk is chunk_frames (F) frames; the window holds window_frames (W) frames including the
+ * current chunk.  Frame f lives in ring slot f mod W, rows [(f mod W)*T_f, (f mod W + 1)*T_f) of the
+ * cache planes; appending frame f evicts frame f - W.
+ */
+#ifndef VMLA_H_
+#define VMLA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VMLA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define VMLA_API __attribute__((visibility("default")))
+#else
+#define VMLA_API
+#endif
+
+typedef enum {
+  VMLA_OK = 0,
+  VMLA_ERR_INVALID_ARG = 1,   /* a null pointer, a bad size, a frame index that does not follow */
+  VMLA_ERR_UNSUPPORTED = 2,   /* sizes the kernels of this dtype do not handle */
+  VMLA_ERR_MISALIGNED = 3,    /* a base pointer that is not 16-byte aligned */
+  VMLA_ERR_CUDA = 4,          /* a CUDA runtime/driver error (detail has the CUDA error text) */
+  VMLA_ERR_TIMEOUT = 5        /* a bounded device-side wait ran out (from vmla_device_status) */
+} vmla_status;
+
+typedef enum { VMLA_BF16 = 0, VMLA_F32 = 1 } vmla_dtype;
+
+/* Layer geometry.  d_h = d_nope + d_rope is the per-head query/key width of the equivalent dense
+ * layer; d_v is the per-head value width.  rope_pairs_t + rope_pairs_h + rope_pairs_w must equal
+ * d_rope / 2 (3D-RoPE pair split over frame, row and column).  softmax_scale <= 0 selects
+ * 1 / sqrt(d_nope + d_rope). */
+typedef struct {
+  int32_t dim, n_heads, d_nope, d_rope, d_c, d_v;
+  int32_t grid_h, grid_w, chunk_frames, window_frames;
+  int32_t rope_pairs_t, rope_pairs_h, rope_pairs_w;
+  float rope_theta;
+  float softmax_scale;
+  int32_t dtype; /* vmla_dtype */
+} vmla_config;
+
+/* The latent cache of one layer: two planes of window_frames*T_f rows per batch element,
+ *   c   [batch, W*T_f, d_c]     the content latents c^KV_t,
+ *   k_r [batch, W*T_f, d_rope]  the rotated positional keys k^R_t.
+ * frames_written counts the frames appended so far (owned by the caller, advanced by
+ * vmla_compress_append).  Rows of slots that were never written are never read. */
+typedef struct {
+  void* c;
+  void* k_r;
+  int32_t batch;
+  int32_t reserved;
+  int64_t frames_written;
+} vmla_cache;
+
+/* The dense per-head cache of the comparison layer: k [batch, W*T_f, n_heads, d_h] and
+ * v [batch, W*T_f, n_heads, d_v], same ring and frame rules as vmla_cache. */
+typedef struct {
+  void* k;
+  void* v;
+  int32_t batch;
+  int32_t reserved;
+  int64_t frames_written;
+} vmla_dense_cache;
+
+/* Compress one chunk into the latent cache (VideoMLA, Method item 1 "shared low-rank content latent"
+ * and item 3 "decoupled 3D-RoPE"; sliding window: abstract and Problem definition).
+ *   x        [batch, F*T_f, dim]          token features of frames first_frame .. first_frame+F-1
+ *   w_dkv_kr [d_c + d_rope, dim]          rows 0..d_c-1 = W^KV_down, rows d_c.. = W^KR
+ * For every token: c = W^KV_down x, k^R = RoPE3D(W^KR x) at the token's (frame, row, column), both
+ * rounded to the storage type and written to its ring row.  first_frame must equal
+ * cache->frames_written; on success cache->frames_written += F. */
+VMLA_API vmla_status vmla_compress_append(const vmla_config* cfg, const void* x, const void* w_dkv_kr,
+                                 int64_t first_frame, vmla_cache* cache, void* stream);
+
+/* Absorbed query (VideoMLA, Method item 2 "on-demand reconstruction" with W^K_up folded into the
+ * query; item 3 for the rotated part).
+ *   q_nope [batch, Nq, n_heads, d_nope], q_rope [batch, Nq, n_heads, d_rope],
+ *   w_uk   [n_heads, d_nope, d_c]  (W^K_up,h maps c to the head's content key),
+ *   q_abs  [batch, Nq, n_heads, d_c + d_rope]  output rows [q~_h ; RoPE3D(q^rope_h)],
+ * with Nq = n_query_chunks*F*T_f tokens of frames first_frame.. (positions of the query tokens). */
+VMLA_API vmla_status vmla_absorb_q(const vmla_config* cfg, int32_t batch, int32_t n_query_chunks,
+                          const void* q_nope, const void* q_rope, const void* w_uk,
+                          int64_t first_frame, void* q_abs, void* stream);
+
+/* Latent attention over the cache (VideoMLA, Method items 2-3; block-causal window: abstract and
+ * Problem definition).  Query token n of the call belongs to chunk k = n / (F*T_f) whose frames end at
+ * hi_k = first_frame + (k+1)*F; it sees the cached keys of frames [max(0, hi_k - W), hi_k):
+ * bidirectional inside its chunk, causal across chunks.  Per (n, h):
+ *   s_t = scale*(q~ . c_t + q^R . k^R_t),  p = softmax(s),  out_latent = sum_t p_t c_t,
+ *   lse = log(sum_t exp(s_t))  (natural log; lse may be NULL).
+ *   q_abs [batch, Nq, n_heads, d_c + d_rope] -> out_latent [batch, Nq, n_heads, d_c], lse [batch, Nq, n_heads].
+ * Requires every needed frame to be in the window: hi_last <= frames_written, and if
+ * frames_written > W then n_query_chunks == 1 and hi_last == frames_written. */
+VMLA_API vmla_status vmla_latent_attention(const vmla_config* cfg, const void* q_abs, const vmla_cache* cache,
+                                  int64_t first_frame, int32_t n_query_chunks, void* out_latent,
+                                  float* lse, void* stream);
+
+/* Value up-projection applied once to the attention-weighted latent (VideoMLA, Method item 2):
+ *   out[b, n, h, :] = W^V_up,h out_latent[b, n, h, :]
+ *   out_latent [batch, n_tokens, n_heads, d_c], w_uv [n_heads, d_v, d_c], out [batch, n_tokens, n_heads, d_v]. */
+VMLA_API vmla_status vmla_value_up(const vmla_config* cfg, int32_t batch, int64_t n_tokens,
+                          const void* out_latent, const void* w_uv, void* out, void* stream);
+
+/* ---- Dense per-head comparison layer (the layout VideoMLA replaces: Problem definition, and
+ *      Method item 4's 2*n_h*d_h scalars per token). ---- */
+
+/* Pack the dense query q [batch, Nq, n_heads, d_h] = [q^nope ; RoPE3D(q^rope)] per head. */
+VMLA_API vmla_status vmla_rope_q(const vmla_config* cfg, int32_t batch, int32_t n_query_chunks,
+                        const void* q_nope, const void* q_rope, int64_t first_frame, void* q,
+                        void* stream);
+
+/* Project one chunk to dense per-head keys and values and append them to the dense ring:
+ *   x [batch, F*T_f, dim], w_kv [n_heads*(d_h + d_v), dim]: rows h*d_h .. h*d_h+d_h-1 give head h's key
+ *   (its last d_rope entries are rotated by 3D-RoPE), rows n_heads*d_h + h*d_v .. give head h's value.
+ * first_frame must equal cache->frames_written; on success cache->frames_written += F. */
+VMLA_API vmla_status vmla_dense_append(const vmla_config* cfg, const void* x, const void* w_kv,
+                              int64_t first_frame, vmla_dense_cache* cache, void* stream);
+
+/* Dense multi-head attention with the same window / block-causal rule as vmla_latent_attention.
+ *   q [batch, Nq, n_heads, d_h] -> out [batch, Nq, n_heads, d_v], lse [batch, Nq, n_heads] (or NULL). */
+VMLA_API vmla_status vmla_dense_mha(const vmla_config* cfg, const void* q, const vmla_dense_cache* cache,
+                           int64_t first_frame, int32_t n_query_chunks, void* out, float* lse,
+                           void* stream);
+
+/* ---- Utilities ---- */
+
+/* Host-only check of the window rule of vmla_latent_attention / vmla_dense_mha for a cache holding
+ * frames_written frames: VMLA_OK if every frame that query chunks first_frame.. need is still in the
+ * window, else VMLA_ERR_INVALID_ARG (with a detail text).  Launches nothing. */
+VMLA_API vmla_status vmla_check_attention_window(const vmla_config* cfg, int64_t frames_written,
+                                                 int64_t first_frame, int32_t n_query_chunks);
+
+/* Synchronise `stream`, then read and clear the device status word of the current device:
+ * *code = 0 if no device-side wait ran out since the last call, else a nonzero code naming the wait.
+ * Returns VMLA_ERR_TIMEOUT when *code != 0. */
+VMLA_API vmla_status vmla_device_status(void* stream, int32_t* code);
+
+/* Bytes of one layer's cache for `batch` sequences at a full window: latent (d_c + d_rope per token)
+ * and dense (n_heads*(d_h + d_v) per token), in the storage type of cfg->dtype.  -1 on a bad cfg. */
+VMLA_API int64_t vmla_latent_cache_bytes(const vmla_config* cfg, int32_t batch);
+VMLA_API int64_t vmla_dense_cache_bytes(const vmla_config* cfg, int32_t batch);
+
+/* Number of kernels the library has launched in this process (all entry points, all devices). */
+VMLA_API int64_t vmla_launch_count(void);
+
+VMLA_API const char* vmla_status_string(vmla_status s);
+VMLA_API const char* vmla_last_error_detail(void);
+VMLA_API int32_t vmla_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VMLA_H_ */

@@ -147,11 +147,14 @@ def reconstruct_kv(c: np.ndarray, k_r: np.ndarray, w_uk: np.ndarray, w_uv: np.nd
     k_{t,h} = [W^K_up,h c_t ; k^R_t] (d_nope + d_rope), v_{t,h} = W^V_up,h c_t (d_v).
     c [T, d_c], k_r [T, d_rope], w_uk [H, d_nope, d_c], w_uv [H, d_v, d_c] -> k [T, H, d_h], v [T, H, d_v]."""
     c = np.asarray(c, F64)
+    k_r = np.asarray(k_r, F64)
     n_heads = w_uk.shape[0]
-    k_nope = np.einsum('hnc,tc->thn', np.asarray(w_uk, F64), c)
-    k_rope = np.broadcast_to(np.asarray(k_r, F64)[:, None, :], (c.shape[0], n_heads, k_r.shape[-1]))
-    k = np.concatenate([k_nope, k_rope], axis=-1)
-    v = np.einsum('hvc,tc->thv', np.asarray(w_uv, F64), c)
+    k = np.empty((c.shape[0], n_heads, w_uk.shape[1] + k_r.shape[-1]), dtype=F64)
+    v = np.empty((c.shape[0], n_heads, w_uv.shape[1]), dtype=F64)
+    for h in range(n_heads):
+        k[:, h, :w_uk.shape[1]] = c @ np.asarray(w_uk[h], F64).T
+        k[:, h, w_uk.shape[1]:] = k_r
+        v[:, h, :] = c @ np.asarray(w_uv[h], F64).T
     return k, v
 
 
@@ -198,9 +201,10 @@ def _masked_softmax(s: np.ndarray, mask: np.ndarray):
 def mha(q: np.ndarray, k: np.ndarray, v: np.ndarray, mask: np.ndarray, scale: float):
     """Textbook per-head softmax attention.  q [N, H, d], k [T, H, d], v [T, H, d_v], mask [N, T]
     -> (o [N, H, d_v], lse [N, H], p [N, H, T])."""
-    s = np.einsum('nhd,thd->nht', np.asarray(q, F64), np.asarray(k, F64)) * scale
+    q, k, v = np.asarray(q, F64), np.asarray(k, F64), np.asarray(v, F64)
+    s = np.stack([q[:, h, :] @ k[:, h, :].T for h in range(q.shape[1])], axis=1) * scale
     p, lse = _masked_softmax(s, mask[:, None, :])
-    o = np.einsum('nht,thv->nhv', p, np.asarray(v, F64))
+    o = np.stack([p[:, h, :] @ v[:, h, :] for h in range(q.shape[1])], axis=1)
     return o, lse, p
 
 
@@ -211,11 +215,11 @@ def latent_attention(q_abs: np.ndarray, c: np.ndarray, k_r: np.ndarray, mask: np
     q_abs [N, H, d_c + d_rope], c [T, d_c], k_r [T, d_rope], mask [N, T]
     -> (o_latent [N, H, d_c], lse [N, H])."""
     q_abs = np.asarray(q_abs, F64)
+    c, k_r = np.asarray(c, F64), np.asarray(k_r, F64)
     d_c = c.shape[-1]
-    s = (np.einsum('nhc,tc->nht', q_abs[..., :d_c], np.asarray(c, F64))
-         + np.einsum('nhr,tr->nht', q_abs[..., d_c:], np.asarray(k_r, F64))) * scale
+    s = (q_abs[..., :d_c] @ c.T + q_abs[..., d_c:] @ k_r.T) * scale        # [N, H, T]
     p, lse = _masked_softmax(s, mask[:, None, :])
-    return np.einsum('nht,tc->nhc', p, np.asarray(c, F64)), lse
+    return p @ c, lse
 
 
 def value_up(o_latent: np.ndarray, w_uv: np.ndarray) -> np.ndarray:
@@ -274,6 +278,6 @@ def layer_reference(hist: History, q_nope, q_rope, w_uk, w_uv, *, first_frame, q
     mask = visible(hi, hist.frames, window_frames)
     k, v = reconstruct_kv(hist.c, hist.k_r, w_uk, w_uv)
     o, lse, p = mha(q, k, v, mask, scale)
-    o_latent = np.einsum('nht,tc->nhc', p, hist.c)
+    o_latent = p @ hist.c
     q_abs = absorbed_query(np.asarray(q_nope, F64)[rows], q_r, w_uk)
     return {"o": o, "o_latent": o_latent, "lse": lse, "q_abs": q_abs, "mask": mask}

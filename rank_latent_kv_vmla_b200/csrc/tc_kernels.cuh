@@ -1,0 +1,45 @@
+// bf16 path of libvmla: tensor-core kernels (tcgen05 / TMEM / TMA on sm_100a).
+#pragma once
+
+#include "vmla_internal.cuh"
+
+namespace vmla {
+
+// Reason text of the last tc_check_* refusal (thread-local).
+const char* tc_last_reason();
+
+vmla_status tc_check_compress(const vmla_config& cfg);
+cudaError_t tc_compress_append(const vmla_config& cfg, int batch, const void* x, const void* w,
+                               const FrameGeom& g, const RopeTable& rt, void* c, void* k_r,
+                               cudaStream_t st);
+
+vmla_status tc_check_absorb(const vmla_config& cfg);
+cudaError_t tc_absorb_q(const vmla_config& cfg, int batch, int64_t nq, const void* q_nope,
+                        const void* q_rope, const void* w_uk, const FrameGeom& g, const RopeTable& rt,
+                        void* q_abs, cudaStream_t st);
+
+vmla_status tc_check_latent_attention(const vmla_config& cfg);
+cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, const void* q_abs,
+                                const void* c, const void* k_r, int64_t cap, int64_t valid_rows,
+                                const FrameGeom& g, float scale, void* out, float* lse, int* status,
+                                cudaStream_t st);
+
+vmla_status tc_check_value_up(const vmla_config& cfg);
+cudaError_t tc_value_up(const vmla_config& cfg, int batch, int64_t n_tokens, const void* o_lat,
+                        const void* w_uv, void* out, cudaStream_t st);
+
+cudaError_t tc_rope_q(const vmla_config& cfg, int batch, int64_t nq, const void* q_nope,
+                      const void* q_rope, const FrameGeom& g, const RopeTable& rt, void* q,
+                      cudaStream_t st);
+
+vmla_status tc_check_dense_append(const vmla_config& cfg);
+cudaError_t tc_dense_append(const vmla_config& cfg, int batch, const void* x, const void* w_kv,
+                            const FrameGeom& g, const RopeTable& rt, void* k, void* v,
+                            cudaStream_t st);
+
+vmla_status tc_check_dense_mha(const vmla_config& cfg);
+cudaError_t tc_dense_mha(const vmla_config& cfg, int batch, int64_t nq, const void* q, const void* k,
+                         const void* v, int64_t cap, int64_t valid_rows, const FrameGeom& g,
+                         float scale, void* out, float* lse, int* status, cudaStream_t st);
+
+}  // namespace vmla

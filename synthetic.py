@@ -72,11 +72,11 @@ def draw_dense_weights(cfg: VmlaConfig, seed: int) -> torch.Tensor:
     return _randn(g, (rows, cfg.dim), cfg.dim ** -0.5, storage_dtype(cfg))
 
 
-def draw_dense_queries(cfg: VmlaConfig, batch: int, seed: int, n_query_chunks: int = 1):
-    """q^nope and q^rope for the dense comparison layer (same shapes as the latent layer's)."""
+def draw_queries(cfg: VmlaConfig, batch: int, seed: int, n_query_chunks: int = 1, q_gain: float = 1.0):
+    """A fresh query set q^nope [B, Nq, n_h, d_nope], q^rope [B, Nq, n_h, d_rope], N(0, q_gain^2)."""
     g = torch.Generator().manual_seed(int(seed))
     dt = storage_dtype(cfg)
     nq = n_query_chunks * cfg.chunk_tokens
-    q_nope = _randn(g, (batch, nq, cfg.n_heads, cfg.d_nope), 1.0, dt)
-    q_rope = _randn(g, (batch, nq, cfg.n_heads, cfg.d_rope), 1.0, dt)
+    q_nope = _randn(g, (batch, nq, cfg.n_heads, cfg.d_nope), q_gain, dt)
+    q_rope = _randn(g, (batch, nq, cfg.n_heads, cfg.d_rope), q_gain, dt)
     return q_nope, q_rope

@@ -1,0 +1,127 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI and the float64 oracle
+on the same seeded inputs, and compare at the stated tolerances.
+
+Tolerances (per output tensor): bf16 storage with fp32 accumulation needs
+max|err| <= 1e-2 * max|ref| and rel-L2 <= 5e-3; the fp32 path needs rel-L2 <= 1e-5.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import vmla_oracle as O
+from rank_latent_kv_vmla_b200.config import VMLA_BF16, VMLA_F32, VmlaConfig, TINY, WAN
+import synthetic
+
+# A mid-size bf16 layer with the Wan head shapes: 60 tokens/frame, 2-frame chunks, 5-frame window.
+# 120 query tokens x 4 heads = 480 query rows (3.75 tiles of 128) and 300 keys (2.3 tiles of 128).
+MID = VmlaConfig(dim=512, n_heads=4, d_nope=96, d_rope=32, d_c=192, d_v=128, grid_h=6, grid_w=10,
+                 chunk_frames=2, window_frames=5, rope_pairs_t=6, rope_pairs_h=5, rope_pairs_w=5,
+                 dtype=VMLA_BF16)
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu").double().numpy()
+
+
+def pairs(cfg: VmlaConfig):
+    return (cfg.rope_pairs_t, cfg.rope_pairs_h, cfg.rope_pairs_w)
+
+
+def hist_kwargs(cfg: VmlaConfig):
+    return dict(d_c=cfg.d_c, d_rope=cfg.d_rope, chunk_frames=cfg.chunk_frames, grid_h=cfg.grid_h,
+                grid_w=cfg.grid_w, pairs=pairs(cfg), theta=cfg.rope_theta)
+
+
+def errors(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), "non-finite values in the GPU output"
+    err = got - ref
+    rel_l2 = float(np.linalg.norm(err) / max(np.linalg.norm(ref), 1e-300))
+    max_ratio = float(np.max(np.abs(err)) / max(np.max(np.abs(ref)), 1e-300))
+    return rel_l2, max_ratio
+
+
+def assert_close(got, ref, cfg: VmlaConfig, what: str):
+    rel_l2, max_ratio = errors(got, ref)
+    if cfg.dtype == VMLA_BF16:
+        assert max_ratio <= 1e-2 and rel_l2 <= 5e-3, \
+            f"{what}: max|err|/max|ref| = {max_ratio:.3e}, rel-L2 = {rel_l2:.3e}"
+    else:
+        assert rel_l2 <= 1e-5, f"{what}: rel-L2 = {rel_l2:.3e}"
+    return rel_l2, max_ratio
+
+
+def round_to(cfg: VmlaConfig, a: np.ndarray) -> torch.Tensor:
+    """Round a float64 array to the storage type (round-to-nearest-even via torch)."""
+    return torch.from_numpy(np.ascontiguousarray(a)).to(synthetic.storage_dtype(cfg))
+
+
+class OracleLayer:
+    """Float64 oracle state of one layer: the full history of every batch element."""
+
+    def __init__(self, cfg: VmlaConfig, inp: synthetic.LayerInputs, batch: int):
+        self.cfg = cfg
+        self.inp = inp
+        self.batch = batch
+        self.w = f64(inp.w_dkv_kr)
+        self.w_uk = f64(inp.w_uk)
+        self.w_uv = f64(inp.w_uv)
+        self.hist = [O.History(cfg.d_c, cfg.d_rope) for _ in range(batch)]
+        self.frames_written = 0
+
+    def append(self, x: torch.Tensor):
+        cfg = self.cfg
+        pos = O.token_positions(self.frames_written, cfg.chunk_tokens, cfg.grid_h, cfg.grid_w)
+        xs = f64(x)
+        for b in range(self.batch):
+            c, k_r = O.compress(xs[b], self.w, cfg.d_c, pos, pairs(cfg), cfg.rope_theta)
+            self.hist[b].append(c, k_r, pos[:, 0])
+        self.frames_written += cfg.chunk_frames
+
+    def ring(self, b: int):
+        cfg = self.cfg
+        c, written = O.ring_from_history(self.hist[b].c, self.frames_written, cfg.window_frames,
+                                         cfg.tokens_per_frame)
+        k_r, _ = O.ring_from_history(self.hist[b].k_r, self.frames_written, cfg.window_frames,
+                                     cfg.tokens_per_frame)
+        return c, k_r, written
+
+    def q_abs(self, q_nope: torch.Tensor, q_rope: torch.Tensor, first_frame: int):
+        cfg = self.cfg
+        nq = q_nope.shape[1]
+        pos = O.token_positions(first_frame, nq, cfg.grid_h, cfg.grid_w)
+        out = []
+        for b in range(q_nope.shape[0]):
+            qr = O.rotate_query(f64(q_rope[b]), pos, pairs(cfg), cfg.rope_theta)
+            out.append(O.absorbed_query(f64(q_nope[b]), qr, self.w_uk))
+        return np.stack(out)
+
+    def reference(self, b: int, q_nope, q_rope, first_frame: int, rows=None):
+        cfg = self.cfg
+        nq = q_nope.shape[1]
+        rows = np.arange(nq) if rows is None else np.asarray(rows)
+        return O.layer_reference(self.hist[b], f64(q_nope[b]), f64(q_rope[b]), self.w_uk, self.w_uv,
+                                 first_frame=first_frame, query_rows=rows,
+                                 chunk_frames=cfg.chunk_frames, window_frames=cfg.window_frames,
+                                 grid_h=cfg.grid_h, grid_w=cfg.grid_w, pairs=pairs(cfg),
+                                 theta=cfg.rope_theta, scale=cfg.scale)
+
+    def key_frames_of_ring(self):
+        """Frame held by each ring row (-1 if unwritten)."""
+        cfg = self.cfg
+        return np.repeat([O.frame_of_slot(s, self.frames_written, cfg.window_frames)
+                          for s in range(cfg.window_frames)], cfg.tokens_per_frame)
+
+
+def dense_weights_from_latent(inp: synthetic.LayerInputs, cfg: VmlaConfig) -> np.ndarray:
+    """Dense per-head K/V weights that make the dense layer equal to the latent one:
+    key rows of head h = [W^K_up,h W^KV_down ; W^KR], value rows = W^V_up,h W^KV_down (float64)."""
+    w = f64(inp.w_dkv_kr)
+    w_dkv, w_kr = w[:cfg.d_c], w[cfg.d_c:]
+    w_uk, w_uv = f64(inp.w_uk), f64(inp.w_uv)
+    keys = [np.concatenate([w_uk[h] @ w_dkv, w_kr]) for h in range(cfg.n_heads)]
+    vals = [w_uv[h] @ w_dkv for h in range(cfg.n_heads)]
+    return np.concatenate(keys + vals)

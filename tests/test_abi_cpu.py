@@ -1,0 +1,119 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol its header declares, and
+rejects bad arguments on the host before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from rank_latent_kv_vmla_b200.config import TINY, WAN, VMLA_F32
+from rank_latent_kv_vmla_b200 import vmla as V
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "vmla.h")
+FAKE = 0x10000          # a 16-byte aligned non-null address: never dereferenced on these paths
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"VMLA_API[^;(]*?\b(vmla_\w+)\s*\(", text)))
+
+
+def test_header_symbols_exported():
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(V.LIB, n), n
+        assert n in V.EXPORTED
+    assert V.LIB.vmla_abi_version() == 1
+
+
+def test_status_strings():
+    assert V.LIB.vmla_status_string(0) == b"ok"
+    assert V.LIB.vmla_status_string(5) == b"device wait timed out"
+
+
+def test_cache_bytes_arithmetic():
+    # 448 B vs 6144 B per token per layer (bf16), 7.29% of the dense layout
+    tok = WAN.window_tokens
+    assert V.latent_cache_bytes(WAN, 1) == tok * 224 * 2
+    assert V.dense_cache_bytes(WAN, 1) == tok * 3072 * 2
+    assert V.latent_cache_bytes(WAN, 8) == 8 * 14_676_480
+    assert abs(V.latent_cache_bytes(WAN, 1) / V.dense_cache_bytes(WAN, 1) - 224 / 3072) < 1e-12
+    assert V.latent_cache_bytes(TINY, 1) == TINY.window_tokens * (TINY.d_c + TINY.d_rope) * 4
+
+
+def _cache(frames_written=0, batch=1, c=FAKE, k=FAKE):
+    return V.CCache(c, k, batch, 0, frames_written)
+
+
+def _status(fn, *args):
+    st = fn(*args)
+    return st, V.LIB.vmla_last_error_detail().decode()
+
+
+def test_bad_configs_rejected():
+    for bad in (TINY.replace(d_rope=7, rope_pairs_w=0), TINY.replace(rope_pairs_t=3),
+                TINY.replace(chunk_frames=4), TINY.replace(dim=0), TINY.replace(dtype=7),
+                TINY.replace(rope_theta=1.0)):
+        cc = V.c_config(bad)
+        st, detail = _status(V.LIB.vmla_compress_append, ctypes.byref(cc), FAKE, FAKE, 0,
+                             ctypes.byref(_cache()), None)
+        assert st == V.VMLA_ERR_INVALID_ARG, (bad, detail)
+    st, _ = _status(V.LIB.vmla_compress_append, None, FAKE, FAKE, 0, ctypes.byref(_cache()), None)
+    assert st == V.VMLA_ERR_INVALID_ARG
+
+
+def test_null_and_misaligned_pointers_rejected():
+    cc = V.c_config(TINY)
+    st, d = _status(V.LIB.vmla_compress_append, ctypes.byref(cc), None, FAKE, 0, ctypes.byref(_cache()), None)
+    assert st == V.VMLA_ERR_INVALID_ARG and "x" in d
+    st, d = _status(V.LIB.vmla_compress_append, ctypes.byref(cc), FAKE + 4, FAKE, 0, ctypes.byref(_cache()), None)
+    assert st == V.VMLA_ERR_MISALIGNED
+    st, d = _status(V.LIB.vmla_value_up, ctypes.byref(cc), 1, 16, FAKE, FAKE + 2, FAKE, None)
+    assert st == V.VMLA_ERR_MISALIGNED and "w_uv" in d
+
+
+def test_append_must_follow_frames_written():
+    cc = V.c_config(TINY)
+    cache = _cache(frames_written=2)
+    st, d = _status(V.LIB.vmla_compress_append, ctypes.byref(cc), FAKE, FAKE, 1, ctypes.byref(cache), None)
+    assert st == V.VMLA_ERR_INVALID_ARG and "follow" in d
+    assert cache.frames_written == 2
+
+
+@pytest.mark.parametrize("fw,first,nchunks,ok", [
+    (0, 0, 1, False),     # empty cache (kv_len = 0)
+    (1, 0, 1, True),
+    (1, 1, 1, False),     # query frames not appended yet
+    (3, 0, 3, True),      # multi-chunk, everything still in the window (W = 3)
+    (4, 3, 1, True),      # window full, newest chunk
+    (4, 2, 1, False),     # an older chunk after eviction
+    (4, 2, 2, False),     # multi-chunk after eviction
+    (3, -1, 1, False),
+    (3, 2, 0, False),
+])
+def test_window_rules(fw, first, nchunks, ok):
+    cc = V.c_config(TINY)
+    st, d = _status(V.LIB.vmla_check_attention_window, ctypes.byref(cc), fw, first, nchunks)
+    assert (st == V.VMLA_OK) == ok, d
+    if not ok:
+        assert st == V.VMLA_ERR_INVALID_ARG
+        # the attention entry points apply the same rule before launching anything
+        cache = _cache(frames_written=fw)
+        st2, _ = _status(V.LIB.vmla_latent_attention, ctypes.byref(cc), FAKE, ctypes.byref(cache), first,
+                         nchunks, FAKE, None, None)
+        assert st2 == V.VMLA_ERR_INVALID_ARG
+        st3, _ = _status(V.LIB.vmla_dense_mha, ctypes.byref(cc), FAKE,
+                         ctypes.byref(V.CDenseCache(FAKE, FAKE, 1, 0, fw)), first, nchunks, FAKE, None, None)
+        assert st3 == V.VMLA_ERR_INVALID_ARG
+
+
+def test_lse_alignment_checked():
+    cc = V.c_config(TINY)
+    st, _ = _status(V.LIB.vmla_latent_attention, ctypes.byref(cc), FAKE, ctypes.byref(_cache(1)), 0, 1,
+                    FAKE, FAKE + 4, None)
+    assert st == V.VMLA_ERR_MISALIGNED
+
+
+def test_device_status_needs_output_pointer():
+    assert V.LIB.vmla_device_status(None, None) == V.VMLA_ERR_INVALID_ARG

@@ -211,7 +211,7 @@ def test_window_mask_matches_streaming_simulation():
 # ------------------------------------------------------------------------------------------------
 def _tiny_history(cfg, seed, n_chunks, q_gain=1.0):
     inp = synthetic.draw_layer(cfg, batch=1, seed=seed, n_chunks=n_chunks, q_gain=q_gain)
-    hist = O.build_history(inp.x_chunks, _f64(inp.w_dkv_kr), 0, **_tiny_kwargs(cfg))
+    hist = O.build_history([_f64(x) for x in inp.x_chunks], _f64(inp.w_dkv_kr), 0, **_tiny_kwargs(cfg))
     return inp, hist
 
 
@@ -361,12 +361,12 @@ def test_streaming_calls_equal_one_block_causal_call():
     cfg = TINY.replace(window_frames=8)
     n_chunks = 4
     inp = synthetic.draw_layer(cfg, batch=1, seed=61, n_chunks=n_chunks, n_query_chunks=n_chunks)
-    hist = O.build_history(inp.x_chunks, _f64(inp.w_dkv_kr), 0, **_tiny_kwargs(cfg))
+    hist = O.build_history([_f64(x) for x in inp.x_chunks], _f64(inp.w_dkv_kr), 0, **_tiny_kwargs(cfg))
     qn, qr = _f64(inp.q_nope[0]), _f64(inp.q_rope[0])
     whole = _ref(cfg, inp, hist, 0, q_nope=qn, q_rope=qr)
     per = cfg.chunk_tokens
     for k in range(n_chunks):
-        part = O.build_history(inp.x_chunks[:k + 1], _f64(inp.w_dkv_kr), 0, **_tiny_kwargs(cfg))
+        part = O.build_history([_f64(x) for x in inp.x_chunks[:k + 1]], _f64(inp.w_dkv_kr), 0, **_tiny_kwargs(cfg))
         one = _ref(cfg, inp, part, k * cfg.chunk_frames, q_nope=qn[k * per:(k + 1) * per],
                    q_rope=qr[k * per:(k + 1) * per])
         np.testing.assert_allclose(whole["o"][k * per:(k + 1) * per], one["o"], rtol=1e-12, atol=1e-14)
