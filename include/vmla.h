@@ -172,6 +172,11 @@ VMLA_API vmla_status vmla_device_status(void* stream, int32_t* code);
 VMLA_API int64_t vmla_latent_cache_bytes(const vmla_config* cfg, int32_t batch);
 VMLA_API int64_t vmla_dense_cache_bytes(const vmla_config* cfg, int32_t batch);
 
+/* Set the bound of every device-side wait of later launches to `ms` milliseconds (default 1000) and
+ * return the previous bound; ms <= 0 only returns the current bound.  A wait that runs out makes the
+ * kernel stop, record a nonzero code for vmla_device_status() and return. */
+VMLA_API int32_t vmla_set_wait_timeout_ms(int32_t ms);
+
 /* Number of kernels the library has launched in this process (all entry points, all devices). */
 VMLA_API int64_t vmla_launch_count(void);
 

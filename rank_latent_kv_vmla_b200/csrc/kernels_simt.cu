@@ -360,6 +360,9 @@ cudaError_t simt_attention(const SimtAttnArgs& a, cudaStream_t st) {
   template cudaError_t simt_attention<T>(const SimtAttnArgs&, cudaStream_t);
 
 VMLA_INSTANTIATE(float)
-VMLA_INSTANTIATE(__nv_bfloat16)
+// bf16 element-wise packing of the dense comparison query (no arithmetic beyond the rotation)
+template cudaError_t simt_rope_q<__nv_bfloat16>(const vmla_config&, int, int64_t, const __nv_bfloat16*,
+                                                const __nv_bfloat16*, const FrameGeom&, const RopeTable&,
+                                                __nv_bfloat16*, cudaStream_t);
 
 }  // namespace vmla

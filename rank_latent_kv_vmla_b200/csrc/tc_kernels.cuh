@@ -1,6 +1,7 @@
 // bf16 path of libvmla: tensor-core kernels (tcgen05 / TMEM / TMA on sm_100a).
 #pragma once
 
+#include "tc_common.cuh"
 #include "vmla_internal.cuh"
 
 namespace vmla {

@@ -21,7 +21,7 @@ VMLA_OK, VMLA_ERR_INVALID_ARG, VMLA_ERR_UNSUPPORTED, VMLA_ERR_MISALIGNED, VMLA_E
 
 EXPORTED = ("vmla_compress_append", "vmla_absorb_q", "vmla_latent_attention", "vmla_value_up",
             "vmla_rope_q", "vmla_dense_append", "vmla_dense_mha", "vmla_device_status",
-            "vmla_check_attention_window",
+            "vmla_check_attention_window", "vmla_set_wait_timeout_ms",
             "vmla_latent_cache_bytes", "vmla_dense_cache_bytes", "vmla_launch_count",
             "vmla_status_string", "vmla_last_error_detail", "vmla_abi_version")
 
@@ -82,6 +82,8 @@ def _load():
     lib.vmla_status_string.restype = ctypes.c_char_p
     lib.vmla_last_error_detail.argtypes = []
     lib.vmla_last_error_detail.restype = ctypes.c_char_p
+    lib.vmla_set_wait_timeout_ms.argtypes = [I32]
+    lib.vmla_set_wait_timeout_ms.restype = I32
     lib.vmla_abi_version.argtypes = []
     lib.vmla_abi_version.restype = I32
     return lib
@@ -288,6 +290,11 @@ def check_attention_window(cfg: VmlaConfig, frames_written: int, first_frame: in
     """Raise VmlaError unless an attention call with these frames would pass the window rule."""
     cc = c_config(cfg)
     check(LIB.vmla_check_attention_window(ctypes.byref(cc), frames_written, first_frame, n_query_chunks))
+
+
+def set_wait_timeout_ms(ms: int) -> int:
+    """Bound (ms) of every device-side wait of later launches; returns the previous bound."""
+    return int(LIB.vmla_set_wait_timeout_ms(int(ms)))
 
 
 def launch_count() -> int:

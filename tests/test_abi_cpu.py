@@ -20,7 +20,7 @@ def _declared():
 
 def test_header_symbols_exported():
     names = _declared()
-    assert len(names) >= 15
+    assert len(names) >= 16
     for n in names:
         assert hasattr(V.LIB, n), n
         assert n in V.EXPORTED
@@ -117,3 +117,10 @@ def test_lse_alignment_checked():
 
 def test_device_status_needs_output_pointer():
     assert V.LIB.vmla_device_status(None, None) == V.VMLA_ERR_INVALID_ARG
+
+
+def test_wait_timeout_setting():
+    old = V.set_wait_timeout_ms(0)
+    assert old == 1000
+    assert V.set_wait_timeout_ms(250) == 1000
+    assert V.set_wait_timeout_ms(old) == 250
