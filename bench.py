@@ -41,7 +41,7 @@ FLUSH_BYTES = 512 << 20   # > 126 MB L2
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--batch", type=int, default=1, help="sequences per GPU")
     ap.add_argument("--impl", default="vmla", choices=["vmla", "reference"])
@@ -194,44 +194,70 @@ def max_over_ranks(x: float, world: int) -> float:
 # ------------------------------------------------------------------------------------------------
 # CPU oracle timing (cpu_baseline leg and --impl reference)
 # ------------------------------------------------------------------------------------------------
-def oracle_sample(cfg, batch, seed, n_rows):
-    """Time the oracle's layer step on a bounded sample: compress the new chunk, then the
-    non-absorbed attention of ``n_rows`` query tokens (all heads) over the full window."""
-    from oracle import vmla_oracle as O
-    import synthetic
-    inp = synthetic.draw_layer(cfg, batch=1, seed=seed, n_chunks=cfg.window_frames // cfg.chunk_frames)
-    xs = [x.double().numpy() for x in inp.x_chunks]
-    w = inp.w_dkv_kr.double().numpy()
-    kw = dict(d_c=cfg.d_c, d_rope=cfg.d_rope, chunk_frames=cfg.chunk_frames, grid_h=cfg.grid_h,
-              grid_w=cfg.grid_w, pairs=(cfg.rope_pairs_t, cfg.rope_pairs_h, cfg.rope_pairs_w),
-              theta=cfg.rope_theta)
-    hist = O.build_history(xs[:-1], w, 0, **kw)
-    f0 = (len(xs) - 1) * cfg.chunk_frames
-    qn, qr = inp.q_nope[0].double().numpy(), inp.q_rope[0].double().numpy()
-    rows = np.linspace(0, cfg.chunk_tokens - 1, n_rows).astype(np.int64)
-    t0 = time.perf_counter()
-    pos = O.token_positions(f0, cfg.chunk_tokens, cfg.grid_h, cfg.grid_w)
-    c, k_r = O.compress(xs[-1][0], w, cfg.d_c, pos, kw["pairs"], cfg.rope_theta)
-    hist.append(c, k_r, pos[:, 0])
-    O.layer_reference(hist, qn, qr, inp.w_uk.double().numpy(), inp.w_uv.double().numpy(),
-                      first_frame=f0, query_rows=rows, chunk_frames=cfg.chunk_frames,
-                      window_frames=cfg.window_frames, grid_h=cfg.grid_h, grid_w=cfg.grid_w,
-                      pairs=kw["pairs"], theta=cfg.rope_theta, scale=cfg.scale)
-    return time.perf_counter() - t0
+class OracleStep:
+    """The float64 oracle on a bounded sample of one layer step: a full 21-frame window is built once
+    (untimed); a timed step compresses ``n_rows`` tokens of the new chunk, absorbs their queries and
+    runs latent attention (the plain definition, all heads) and the value up-projection for them."""
+
+    def __init__(self, cfg, seed):
+        from oracle import vmla_oracle as O
+        import synthetic
+        self.O, self.cfg = O, cfg
+        n_chunks = cfg.window_frames // cfg.chunk_frames
+        inp = synthetic.draw_layer(cfg, batch=1, seed=seed, n_chunks=n_chunks)
+        self.pairs = (cfg.rope_pairs_t, cfg.rope_pairs_h, cfg.rope_pairs_w)
+        self.w = inp.w_dkv_kr.double().numpy()
+        self.w_uk, self.w_uv = inp.w_uk.double().numpy(), inp.w_uv.double().numpy()
+        self.x_new = inp.x_chunks[-1][0].double().numpy()
+        self.qn, self.qr = inp.q_nope[0].double().numpy(), inp.q_rope[0].double().numpy()
+        kw = dict(d_c=cfg.d_c, d_rope=cfg.d_rope, chunk_frames=cfg.chunk_frames, grid_h=cfg.grid_h,
+                  grid_w=cfg.grid_w, pairs=self.pairs, theta=cfg.rope_theta)
+        hist = O.build_history([x.double().numpy() for x in inp.x_chunks], self.w, 0, **kw)
+        self.c, self.k_r, self.frames = hist.c, hist.k_r, hist.frames
+        self.f0 = (n_chunks - 1) * cfg.chunk_frames
+
+    def run(self, n_rows: int) -> float:
+        """Time the sample; the rows go through the oracle in groups of at most 128 (bounded memory)."""
+        rows_all = np.linspace(0, self.cfg.chunk_tokens - 1, n_rows).astype(np.int64)
+        return sum(self._run_rows(rows_all[i:i + 128]) for i in range(0, n_rows, 128))
+
+    def _run_rows(self, rows) -> float:
+        O, cfg = self.O, self.cfg
+        t0 = time.perf_counter()
+        pos = O.token_positions(self.f0, cfg.chunk_tokens, cfg.grid_h, cfg.grid_w)[rows]
+        O.compress(self.x_new[rows], self.w, cfg.d_c, pos, self.pairs, cfg.rope_theta)
+        q_abs = O.absorbed_query(self.qn[rows], O.rotate_query(self.qr[rows], pos, self.pairs, cfg.rope_theta),
+                                 self.w_uk)
+        hi = O.query_chunk_end(self.f0, cfg.chunk_tokens, cfg.chunk_frames, cfg.tokens_per_frame)[rows]
+        mask = O.visible(hi, self.frames, cfg.window_frames)
+        o_lat, _ = O.latent_attention(q_abs, self.c, self.k_r, mask, cfg.scale)
+        O.value_up(o_lat, self.w_uv)
+        return time.perf_counter() - t0
+
+    def size_for(self, seconds: float) -> int:
+        """Rows whose step takes about `seconds` (linear fit t = a + b*n from two probes)."""
+        n1, n2 = 8, 32
+        t1, t2 = self.run(n1), self.run(n2)
+        b = max((t2 - t1) / (n2 - n1), 1e-6)
+        a = max(t1 - b * n1, 0.0)
+        return int(min(self.cfg.chunk_tokens, max(1, (seconds - a) / b)))
+
+
+def _sample_text(cfg, n_rows, t):
+    return (f"float64 NumPy oracle, one Wan-1.3B layer step restricted to {n_rows} of {cfg.chunk_tokens} "
+            f"query tokens: their compression, absorbed queries, latent attention over the full "
+            f"{cfg.window_tokens}-token window (all {cfg.n_heads} heads) and value up-projection; "
+            f"{t:.2f} s; value = those rows' latent-attention flops / time")
 
 
 def cpu_baseline(cfg, target_s):
     cores = len(os.sched_getaffinity(0))
-    probe = 32
-    t_probe = oracle_sample(cfg, 1, 4321, probe)
-    n_rows = int(min(cfg.chunk_tokens, max(probe, probe * target_s / max(t_probe, 1e-3))))
-    t = oracle_sample(cfg, 1, 4321, n_rows)
+    st = OracleStep(cfg, 4321)
+    n_rows = st.size_for(target_s)
+    t = st.run(n_rows)
     flops = attention_flops(cfg, 1) * n_rows / cfg.chunk_tokens
     return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "query_tokens_per_s": n_rows / t,
-            "sample": f"float64 NumPy oracle, one layer step of the Wan-1.3B layer restricted to {n_rows} "
-                      f"of {cfg.chunk_tokens} query tokens (all {cfg.n_heads} heads, full 21-frame window, "
-                      f"non-absorbed K/V materialised), {t:.1f} s; value = those rows' latent-attention flops / time"}
+            "query_tokens_per_s": n_rows / t, "sample": _sample_text(cfg, n_rows, t)}
 
 
 def run_reference(args):
@@ -240,10 +266,13 @@ def run_reference(args):
         return
     cfg = WAN
     cores = len(os.sched_getaffinity(0))
-    n_rows = 48
+    st = OracleStep(cfg, 4321)
+    budget = 150.0                      # seconds for all warm-up + timed steps
+    per_step = min(5.0, budget / max(1, args.steps + args.warmup))
+    n_rows = st.size_for(per_step)
     for _ in range(args.warmup):
-        oracle_sample(cfg, 1, 4321, n_rows)
-    times = [oracle_sample(cfg, 1, 4321, n_rows) for _ in range(args.steps)]
+        st.run(n_rows)
+    times = [st.run(n_rows) for _ in range(args.steps)]
     t = sum(times)
     flops = attention_flops(cfg, 1) * n_rows / cfg.chunk_tokens * args.steps
     val = flops / t / 1e12
@@ -255,8 +284,7 @@ def run_reference(args):
                        "query_tokens": cfg.chunk_tokens, "cached_tokens": cfg.window_tokens},
             "impl": "reference",
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{n_rows} of {cfg.chunk_tokens} query tokens per step (all heads), "
-                                       "float64 NumPy oracle incl. the chunk's compression"},
+                             "sample": _sample_text(cfg, n_rows, t / args.steps) + " (per step)"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

@@ -177,6 +177,12 @@ VMLA_API int64_t vmla_dense_cache_bytes(const vmla_config* cfg, int32_t batch);
  * kernel stop, record a nonzero code for vmla_device_status() and return. */
 VMLA_API int32_t vmla_set_wait_timeout_ms(int32_t ms);
 
+/* Test hook for the bounded-wait path: the next bf16 vmla_latent_attention launch does not load KV
+ * tile `tile` (keys tile*128 .. tile*128+127) of any query tile, so the wait for it runs out, the
+ * kernel winds down without writing its outputs and vmla_device_status() reports a nonzero code.
+ * tile < 0 clears a pending request.  Nothing is faulted; later launches are unaffected. */
+VMLA_API void vmla_debug_drop_kv_tile(int32_t tile);
+
 /* Number of kernels the library has launched in this process (all entry points, all devices). */
 VMLA_API int64_t vmla_launch_count(void);
 

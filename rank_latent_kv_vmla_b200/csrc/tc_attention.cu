@@ -48,6 +48,7 @@ struct AttnParams {
   float* lse;
   int* status;
   uint64_t limit_ns;
+  int drop_kv_tile;      // test hook: this KV tile is never loaded (-1: none)
 };
 
 // Shared-memory plan of one kernel instance.
@@ -135,6 +136,8 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         const int st = j % NST;
         if (j >= NST && !mbar_wait(kv_empty + st, ((j / NST) - 1) & 1, abort_flag, p.status, 1, p.limit_ns))
           break;
+        issued = j + 1;
+        if (j == p.drop_kv_tile) continue;
         uint8_t* stage = sKV + st * P::kStageBytes;
         mbar_arrive_expect_tx(kv_full + st, P::kStageBytes);
         const int krow = j * kBlockN;
@@ -143,13 +146,12 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         if (!V_ALIAS)
           for (int i = 0; i < VB; ++i)
             tma_load_4d(stage + P::kKBytes + i * kBoxBytes, &map_v, kv_full + st, 64 * i, h, krow, b);
-        issued = j + 1;
       }
       if (*abort_flag) {
         // let the copies already issued land before the CTA exits
         mbar_wait(bar_q, 0, &zero_flag, nullptr, 0, p.limit_ns);
         for (int j = (issued > NST ? issued - NST : 0); j < issued; ++j)
-          mbar_wait(kv_full + j % NST, (j / NST) & 1, &zero_flag, nullptr, 0, p.limit_ns);
+          if (j != p.drop_kv_tile) mbar_wait(kv_full + j % NST, (j / NST) & 1, &zero_flag, nullptr, 0, p.limit_ns);
       }
     }
   } else if (warp == 5) {
@@ -226,27 +228,29 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       const bool got = mbar_wait(s_full + bj, (j >> 1) & 1, abort_flag, p.status, 6, p.limit_ns);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      float s[kBlockN];
-      {
-        uint32_t raw[32];
+      // S row of this thread (raw scores): four 32-column TMEM loads, one wait
+      uint32_t sr[kBlockN];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(tmem + lane_base + bj * 128 + c * 32, raw);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(raw[i]) * p.scale_log2;
-        }
-      }
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(tmem + lane_base + bj * 128 + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
+      tmem_ld_wait();
       const int64_t key0 = (int64_t)j * kBlockN;
       if (key0 + kBlockN > kend_first) {
 #pragma unroll
         for (int i = 0; i < kBlockN; ++i)
-          if (key0 + i >= kend) s[i] = -INFINITY;
+          if (key0 + i >= kend) sr[i] = __float_as_uint(-INFINITY);
       }
-      float mt = s[0];
+      // row max as a tree of 8 independent chains (the scale is positive, so it is applied after)
+      float mx[8];
 #pragma unroll
-      for (int i = 1; i < kBlockN; ++i) mt = fmaxf(mt, s[i]);
-      const float m_new = fmaxf(m_ref, mt);
+      for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(sr[i]);
+#pragma unroll
+      for (int i = 8; i < kBlockN; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[i]));
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+      const float m_new = fmaxf(m_ref, mx[0] * p.scale_log2);
       const bool need = m_new > m_ref + kRescaleThreshold;
       if (__any_sync(0xffffffffu, need)) {
         const float alpha = fast_exp2(m_ref - m_new);   // 0 on the first tile
@@ -266,20 +270,30 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         l_sum *= alpha;
         m_ref = m_new;
       }
+      // p = 2^(s * scale*log2(e) - m) (one FFMA + one MUFU.EX2 per score), row sum in 8 chains,
+      // P packed to bf16 pairs over the first 64 columns of this S buffer
+      const float neg_m = -m_ref;
+      float ls[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ls[i] = 0.f;
       uint32_t pk[32];
-      float lsum_tile = 0.f;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = fast_exp2(s[c * 64 + 2 * i] - m_ref);
-          const float p1 = fast_exp2(s[c * 64 + 2 * i + 1] - m_ref);
-          lsum_tile += p0 + p1;
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c * 64 + 2 * i]), p.scale_log2, neg_m));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c * 64 + 2 * i + 1]), p.scale_log2, neg_m));
+          ls[(2 * i) & 7] += p0;
+          ls[(2 * i + 1) & 7] += p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st32(tmem + lane_base + bj * 128 + c * 32, pk);
       }
-      l_sum += lsum_tile;
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) ls[i] += ls[i + w];
+      l_sum += ls[0];
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_ready + bj);
@@ -390,6 +404,7 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
   p.lse = lse;
   p.status = status;
   p.limit_ns = wait_limit_ns();
+  p.drop_kv_tile = take_drop_kv_tile();
   const int n_tiles = batch * p.tiles_per_group;
   switch (cfg.d_c) {
     case 64: return launch_attention<1, 32, 1, true>(m, p, n_tiles, st);
@@ -426,6 +441,7 @@ cudaError_t tc_dense_mha(const vmla_config& cfg, int batch, int64_t nq, const vo
   p.lse = lse;
   p.status = status;
   p.limit_ns = wait_limit_ns();
+  p.drop_kv_tile = -1;
   const int n_tiles = batch * H * p.tiles_per_group;
   return launch_attention<2, 0, 2, false>(m, p, n_tiles, st);
 }

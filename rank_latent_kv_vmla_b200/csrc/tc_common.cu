@@ -11,6 +11,7 @@ namespace vmla {
 namespace {
 
 std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};   // 1 s
+std::atomic<int> g_drop_kv_tile{-1};
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -29,6 +30,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }  // namespace
 
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
+
+int take_drop_kv_tile() { return g_drop_kv_tile.exchange(-1); }
 
 cudaError_t ensure_smem_attr(const void* kernel, int bytes, std::atomic<uint64_t>& done) {
   int dev = 0;
@@ -73,3 +76,5 @@ extern "C" VMLA_API int32_t vmla_set_wait_timeout_ms(int32_t ms) {
   if (ms > 0) vmla::g_wait_limit_ns.store((uint64_t)ms * 1000000ull);
   return (int32_t)old;
 }
+
+extern "C" VMLA_API void vmla_debug_drop_kv_tile(int32_t tile) { vmla::g_drop_kv_tile.store(tile); }

@@ -27,6 +27,9 @@ uint64_t wait_limit_ns();
 // Raise a kernel's dynamic shared-memory limit once per device (bit d of `done` marks device d).
 cudaError_t ensure_smem_attr(const void* kernel, int bytes, std::atomic<uint64_t>& done);
 
+// Test hook of vmla_debug_drop_kv_tile: returns the pending tile index (or -1) and clears it.
+int take_drop_kv_tile();
+
 // Reason of the last refusal by a tc_check_* function (thread-local).
 void set_tc_reason(const char* why);
 

@@ -27,7 +27,6 @@ using bf16 = __nv_bfloat16;
 constexpr int kThreads = 192;
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBK * 2;   // 16 KB
 
 struct GemmShape {
@@ -57,7 +56,7 @@ __device__ __forceinline__ void rope32(const RopeTable& rt, int pair0, int64_t f
 #pragma unroll
   for (int q = 0; q < 16; ++q) {
     float a, b;
-    rope_rotate(rt, pair0 + q, f, i, j, v[2 * q], v[2 * q + 1], &a, &b);
+    rope_rotate_f32(rt, pair0 + q, f, i, j, v[2 * q], v[2 * q + 1], &a, &b);
     v[2 * q] = a;
     v[2 * q + 1] = b;
   }
@@ -137,8 +136,9 @@ struct EpiDense {
   __device__ void finish(int, int64_t) const {}
 };
 
-template <int BN, bool B_MN_MAJOR>
+template <int BN, bool B_MN_MAJOR, int STAGES>
 struct GemmPlan {
+  static constexpr int kStages = STAGES;
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;
@@ -147,11 +147,12 @@ struct GemmPlan {
   static_assert(!B_MN_MAJOR || BN % 64 == 0, "MN-major B is loaded in 64-column boxes");
 };
 
-template <int BN, bool B_MN_MAJOR, class Epi>
+template <int BN, bool B_MN_MAJOR, int STAGES, class Epi>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
             const GemmShape sh, Epi epi) {
-  using PL = GemmPlan<BN, B_MN_MAJOR>;
+  using PL = GemmPlan<BN, B_MN_MAJOR, STAGES>;
+  constexpr int kStages = STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * PL::kStageBytes);
@@ -266,11 +267,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
   }
 }
 
-template <int BN, bool B_MN_MAJOR, class Epi>
-cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmShape& sh, int heads,
-                        const Epi& epi, cudaStream_t st) {
-  using PL = GemmPlan<BN, B_MN_MAJOR>;
-  auto kern = gemm_kernel<BN, B_MN_MAJOR, Epi>;
+template <int BN, bool B_MN_MAJOR, int STAGES, class Epi>
+cudaError_t launch_gemm_st(const CUtensorMap& a, const CUtensorMap& b, const GemmShape& sh, int heads,
+                           const Epi& epi, cudaStream_t st) {
+  using PL = GemmPlan<BN, B_MN_MAJOR, STAGES>;
+  auto kern = gemm_kernel<BN, B_MN_MAJOR, STAGES, Epi>;
   static std::atomic<uint64_t> done{0};
   cudaError_t attr_err = ensure_smem_attr((const void*)kern, PL::kSmemBytes, done);
   if (attr_err != cudaSuccess) return attr_err;
@@ -278,6 +279,15 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmSh
   kern<<<grid, kThreads, PL::kSmemBytes, st>>>(a, b, sh, epi);
   count_launches(1);
   return cudaGetLastError();
+}
+
+// Short reductions (K <= 2 k-tiles per stage ring) use a 2-deep ring so that several CTAs share an SM
+// and one CTA's epilogue overlaps another's loads; long ones (the D = 1536 projections) a 4-deep ring.
+template <int BN, bool B_MN_MAJOR, class Epi>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmShape& sh, int heads,
+                        const Epi& epi, cudaStream_t st) {
+  if (sh.K <= 4 * kBK) return launch_gemm_st<BN, B_MN_MAJOR, 2>(a, b, sh, heads, epi, st);
+  return launch_gemm_st<BN, B_MN_MAJOR, 4>(a, b, sh, heads, epi, st);
 }
 
 }  // namespace

@@ -66,6 +66,21 @@ __device__ __forceinline__ void rope_rotate(const RopeTable& rt, int p, int64_t 
   *rb = a * sf + b * cf;
 }
 
+// Same rotation for bf16 outputs: the angle is formed and reduced to [-pi, pi] in double precision
+// (so large frame indices lose nothing), then its sine and cosine are taken in single precision.
+__device__ __forceinline__ void rope_rotate_f32(const RopeTable& rt, int p, int64_t f, int64_t i,
+                                                int64_t j, float a, float b, float* ra, float* rb) {
+  const int ax = rt.axis[p];
+  const double pos = (double)(ax == 0 ? f : (ax == 1 ? i : j));
+  const double two_pi = 6.283185307179586476925286766559;
+  double ang = pos * rt.inv_freq[p];
+  ang = fma(-two_pi, rint(ang / two_pi), ang);
+  float sf, cf;
+  sincosf((float)ang, &sf, &cf);
+  *ra = a * cf - b * sf;
+  *rb = a * sf + b * cf;
+}
+
 // Device status word (bounded waits that ran out record a nonzero code here).
 int* device_status_ptr();   // address of this device's status word (host side), nullptr on error
 void count_launches(int n);

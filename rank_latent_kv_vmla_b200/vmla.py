@@ -21,7 +21,7 @@ VMLA_OK, VMLA_ERR_INVALID_ARG, VMLA_ERR_UNSUPPORTED, VMLA_ERR_MISALIGNED, VMLA_E
 
 EXPORTED = ("vmla_compress_append", "vmla_absorb_q", "vmla_latent_attention", "vmla_value_up",
             "vmla_rope_q", "vmla_dense_append", "vmla_dense_mha", "vmla_device_status",
-            "vmla_check_attention_window", "vmla_set_wait_timeout_ms",
+            "vmla_check_attention_window", "vmla_set_wait_timeout_ms", "vmla_debug_drop_kv_tile",
             "vmla_latent_cache_bytes", "vmla_dense_cache_bytes", "vmla_launch_count",
             "vmla_status_string", "vmla_last_error_detail", "vmla_abi_version")
 
@@ -82,6 +82,8 @@ def _load():
     lib.vmla_status_string.restype = ctypes.c_char_p
     lib.vmla_last_error_detail.argtypes = []
     lib.vmla_last_error_detail.restype = ctypes.c_char_p
+    lib.vmla_debug_drop_kv_tile.argtypes = [I32]
+    lib.vmla_debug_drop_kv_tile.restype = None
     lib.vmla_set_wait_timeout_ms.argtypes = [I32]
     lib.vmla_set_wait_timeout_ms.restype = I32
     lib.vmla_abi_version.argtypes = []
@@ -295,6 +297,12 @@ def check_attention_window(cfg: VmlaConfig, frames_written: int, first_frame: in
 def set_wait_timeout_ms(ms: int) -> int:
     """Bound (ms) of every device-side wait of later launches; returns the previous bound."""
     return int(LIB.vmla_set_wait_timeout_ms(int(ms)))
+
+
+def debug_drop_kv_tile(tile: int) -> None:
+    """Test hook: the next bf16 latent attention launch skips loading KV tile ``tile`` (its wait runs
+    out and vmla_device_status reports it); tile < 0 clears the request."""
+    LIB.vmla_debug_drop_kv_tile(int(tile))
 
 
 def launch_count() -> int:

@@ -285,3 +285,36 @@ def test_native_kernels_launched(V):
                  _to(inp.w_uk), _to(inp.w_uv), cache)
     torch.cuda.synchronize()
     assert V.launch_count() > before
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(V):
+    """A KV tile that is never loaded makes the consumer's bounded wait run out: the kernel returns,
+    vmla_device_status reports a nonzero code, and the next call on the same context is correct."""
+    cfg = MID
+    inp = synthetic.draw_layer(cfg, batch=1, seed=404, n_chunks=3)
+    cache = V.LatentCache(cfg, 1, device=DEV)
+    for x in inp.x_chunks:
+        f0 = cache.frames_written
+        V.compress_append(cfg, _to(x), _to(inp.w_dkv_kr), cache)
+    q_abs = V.absorb_q(cfg, _to(inp.q_nope), _to(inp.q_rope), _to(inp.w_uk), f0)
+    torch.cuda.synchronize()
+    assert V.device_status() == 0
+    old = V.set_wait_timeout_ms(20)
+    try:
+        V.debug_drop_kv_tile(1)
+        V.latent_attention(cfg, q_abs, cache, f0)
+        torch.cuda.synchronize()
+        code = V.device_status()
+        assert code != 0
+        assert V.device_status() == 0          # reading clears it
+    finally:
+        V.debug_drop_kv_tile(-1)
+        V.set_wait_timeout_ms(old)
+    o_lat, lse = V.latent_attention(cfg, q_abs, cache, f0, want_lse=True)
+    torch.cuda.synchronize()
+    assert V.device_status() == 0
+    orc = OracleLayer(cfg, inp, 1)
+    for x in inp.x_chunks:
+        orc.append(x)
+    ref = orc.reference(0, inp.q_nope, inp.q_rope, f0)
+    assert_close(f64(o_lat[0]), ref["o_latent"], cfg, "o_latent after a timed-out launch")
