@@ -163,15 +163,17 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------------
 # Distributed plumbing (one process per GPU; timing collective only)
 # ------------------------------------------------------------------------------------------------
-def dist_setup(n_gpus):
+def dist_setup(backend: str = "nccl"):
+    """One process per GPU (torchrun env).  Returns (rank, world, local_rank)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if world > 1:
         import datetime
         import torch.distributed as dist
         rank = int(os.environ["RANK"])
         local = int(os.environ.get("LOCAL_RANK", rank))
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
         return rank, world, local
     return 0, 1, 0
 
@@ -182,13 +184,24 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device="cuda") -> float:
+    """Largest value over all ranks (the timing collective: every rank calls it once per region)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's inputs: the headline layer's seed for rank 0, distinct per rank."""
+    return 1234 + 1 + 1000 * rank
+
+
+def whole_job_rate(work_per_step: float, steps: int, world: int, max_total_ms: float) -> float:
+    """Work of all ranks (each rank runs its own batch) per second of the slowest rank."""
+    return world * work_per_step * steps / (max_total_ms * 1e-3)
 
 
 # ------------------------------------------------------------------------------------------------
@@ -298,7 +311,7 @@ def main():
         return run_reference(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    rank, world, local = dist_setup(args.gpus)
+    rank, world, local = dist_setup("nccl")
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     from rank_latent_kv_vmla_b200 import vmla as V
@@ -307,7 +320,7 @@ def main():
     cfg = WAN
     B = args.batch
     pk, pk_src = peaks()
-    seed = 1234 + 1 + 1000 * rank
+    seed = rank_seed(rank)
     prefill = cfg.window_frames // cfg.chunk_frames - 1          # 6 chunks: frames 0..17
     inp = synthetic.draw_layer(cfg, batch=B, seed=seed, n_chunks=prefill + N_INPUT_SETS)
     extra_q = [synthetic.draw_queries(cfg, B, seed + 7 + i) for i in range(N_INPUT_SETS)]
@@ -367,8 +380,8 @@ def main():
     assert V.device_status() == 0
 
     f_step = attention_flops(cfg, B)
-    value = world * f_step * args.steps / (total_ms * 1e-3) / 1e12
-    q_tok_s = world * B * cfg.chunk_tokens * args.steps / (total_ms * 1e-3)
+    value = whole_job_rate(f_step, args.steps, world, total_ms) / 1e12
+    q_tok_s = whole_job_rate(B * cfg.chunk_tokens, args.steps, world, total_ms)
     k3_ms = statistics.mean(per_kernel["latent_attention"])
     k3_tflops = f_step / (k3_ms * 1e-3) / 1e12
     kb = kernel_bytes(cfg, B)
