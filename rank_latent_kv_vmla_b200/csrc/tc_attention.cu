@@ -5,14 +5,21 @@
 //    the shared latent; here the reconstruction is folded into the query and applied after the sum);
 //  * the dense per-head comparison layer (d_h = d_v = 128 per head).
 //
-// One CTA owns one tile of 128 query rows and streams every visible KV tile of 128 keys:
-//   warp 4      TMA producer: Q tile once, then KV tiles into an NST-deep shared-memory ring;
+// One CTA owns one tile of 128 query rows and streams every visible KV tile of BN keys:
+//   warp 4      TMA producer: KV tiles into an NST-deep shared-memory ring (and the Q tile when Q
+//               is kept in shared memory);
 //   warp 5      TMEM owner and MMA issuer: S_j = Q K_j^T into one of two TMEM S buffers, then
 //               O += P_{j-1} V_{j-1} with P read from TMEM (it overwrites S_{j-1} as bf16);
-//   warps 0-3   softmax, one thread per query row (TMEM lane): masked running max with a lazy
-//               rescale of O (only when the max grows by more than 2^8), exp2, row sum, P to TMEM;
-//               finally O / l to global memory and the log-sum-exp.
-// The KV ring is released by tcgen05.commit after the P*V MMAs that last read a stage.
+//   warps 0-3   one thread per query row (= TMEM lane): first the Q row into TMEM (when Q is kept
+//               in TMEM), then per tile the softmax: masked running max with a lazy rescale of O (only
+//               when the max grows by more than 2^8), exp2, row sum, P to TMEM; finally O / l to
+//               global memory and the log-sum-exp.  The softmax is issue-bound, so it uses 3-input
+//               max and packed f32x2 FMA / add instructions.
+// Keeping Q in TMEM makes S = Q K^T read only K from shared memory: with Q re-read from shared
+// memory by every MMA, the QK^T MMAs, the P V MMAs and the TMA writes together exceed the shared
+// memory bandwidth and the tensor pipe stalls.  The TMEM budget (512 columns: 2 S buffers, O, Q) then
+// sets BN: 96 keys for d_c = 192, 128 keys for smaller latents and for the dense layer.
+// The KV ring is released by tcgen05.commit after the P V MMAs that last read a stage.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -29,14 +36,11 @@ using namespace sm100;
 
 constexpr int kThreads = 192;          // 6 warps
 constexpr int kBlockM = 128;           // query rows per CTA
-constexpr int kBlockN = 128;           // keys per KV tile
-constexpr int kBoxBytes = kBlockN * 64 * 2;   // one [128 x 64] bf16 box (16 KB)
-constexpr int kRopeBoxBytes = kBlockN * 32 * 2;  // one [128 x 32] bf16 box (8 KB)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 256;       // O accumulator columns start here (S buffers at 0 and 128)
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct AttnParams {
+  const void* q;         // query rows (used when Q is kept in TMEM)
   int rows_per_b;        // query rows per batch element (latent: Nq*H, dense: Nq)
   int tiles_per_group;   // query tiles per (batch[, head]) group
   int heads;             // dense: heads per token (tile groups are (b, h)); latent: n = row / heads
@@ -51,41 +55,66 @@ struct AttnParams {
   int drop_kv_tile;      // test hook: this KV tile is never loaded (-1: none)
 };
 
-// Shared-memory plan of one kernel instance.
-template <int KB, int KR, int VB, bool V_ALIAS>
+// Compile-time plan of one kernel instance.
+//   KB    64-column boxes of the key tile from the first key plane (c, or dense K)
+//   KR    width of the rope box (0 or 32, 64-byte swizzle)
+//   VB    64-column boxes of the value tile (V = the first VB key boxes when V_ALIAS)
+//   BN    keys per KV tile;  NS  TMEM S buffers (the MMA runs NS - 1 tiles ahead of P V)
+//   Q_TMEM  whether Q lives in TMEM (the A operand of S = Q K^T) or in shared memory
+//   ONES  V is extended by 16 columns of ones in shared memory, so that the P V MMA also produces
+//         the row sum of P in O's column DV (the softmax then needs no add chains)
+template <int KB, int KR, int VB, bool V_ALIAS, int BN, int NS, bool Q_TMEM, bool ONES>
 struct Plan {
-  static constexpr int kQBytes = KB * kBoxBytes + (KR ? kRopeBoxBytes : 0);
-  static constexpr int kKBytes = KB * kBoxBytes + (KR ? kRopeBoxBytes : 0);
-  static constexpr int kVBytes = V_ALIAS ? 0 : VB * kBoxBytes;
-  static constexpr int kStageBytes = kKBytes + kVBytes;
-  static constexpr int kBudget = 232448 - 1024 - 256;
-  static constexpr int kStages = ((kBudget - kQBytes) / kStageBytes) >= 4 ? 4 : ((kBudget - kQBytes) / kStageBytes);
-  static constexpr int kSmemBytes = kQBytes + kStages * kStageBytes + 256 + 1024;
+  static constexpr int kDQK = 64 * KB + KR;
   static constexpr int kDV = 64 * VB;
-  static_assert(kStages >= 2, "shared memory too small for two KV stages");
-  static_assert(kTmemO + kDV <= kTmemCols, "TMEM budget");
+  static constexpr int kNPV = kDV + (ONES ? 16 : 0);     // N of the P V MMA
+  static constexpr int kBox = BN * 128;                 // [BN x 64] bf16 box, 128-byte swizzle
+  static constexpr int kRopeBox = BN * 64;              // [BN x 32] bf16 box, 64-byte swizzle
+  static constexpr int kQBytes = Q_TMEM ? 0 : (KB * kBlockM * 128 + (KR ? kBlockM * 64 : 0));
+  // stage layout: K boxes | V boxes (unless aliased) | ones box | rope box
+  static constexpr int kVOff = V_ALIAS ? 0 : KB * kBox;
+  static constexpr int kOnesOff = kVOff + VB * kBox;
+  static constexpr int kRopeOff = (V_ALIAS && !ONES) ? KB * kBox : kOnesOff + (ONES ? kBox : 0);
+  static constexpr int kStageRaw = kRopeOff + (KR ? kRopeBox : 0);
+  static constexpr int kStageBytes = (kStageRaw + 1023) / 1024 * 1024;
+  static constexpr int kLoadBytes = KB * kBox + (V_ALIAS ? 0 : VB * kBox) + (KR ? kRopeBox : 0);
+  static constexpr int kAuxBytes = 512;                 // barriers
+  static constexpr int kBudget = 232448 - 1024 - kAuxBytes;
+  static constexpr int kFit = (kBudget - kQBytes) / kStageBytes;
+  static constexpr int kStages = kFit >= 6 ? 6 : kFit;
+  static constexpr int kSmemBytes = kQBytes + kStages * kStageBytes + kAuxBytes + 1024;
+  // TMEM columns: S buffers [b*BN, (b+1)*BN) for b < NS, O [NS*BN, NS*BN + NPV), Q after O
+  static constexpr uint32_t kTmemO = NS * BN;
+  static constexpr uint32_t kTmemQ = NS * BN + kNPV;
+  static_assert(kStages >= NS, "shared memory too small for the KV ring");
+  static_assert(kTmemQ + (Q_TMEM ? kDQK / 2 : 0) <= kTmemCols, "TMEM budget");
+  static_assert(BN % 32 == 0 && BN <= 128 && NS >= 2 && NS <= 3, "tile shape");
+  static_assert(kDV % 32 == 0 && (kDQK / 2) % 8 == 0, "row chunks");
+  static_assert(!ONES || Q_TMEM, "the ones box is filled by the warps that also write Q into TMEM");
+  static_assert(kNPV <= 256 && kNPV % 16 == 0, "P V MMA shape");
 };
 
-template <int KB, int KR, int VB, bool V_ALIAS>
+template <int KB, int KR, int VB, bool V_ALIAS, int BN, int NS, bool Q_TMEM, bool ONES>
 __global__ void __launch_bounds__(kThreads, 1)
 attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_qr,
                  const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_kr,
                  const __grid_constant__ CUtensorMap map_v, const AttnParams p) {
-  using P = Plan<KB, KR, VB, V_ALIAS>;
-  constexpr int NST = P::kStages;
-  constexpr int DV = P::kDV;
+  using PL = Plan<KB, KR, VB, V_ALIAS, BN, NS, Q_TMEM, ONES>;
+  constexpr int NST = PL::kStages;
+  constexpr int DV = PL::kDV;
+  constexpr int DQK = PL::kDQK;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sKV = smem + P::kQBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NST * P::kStageBytes);
-  uint64_t* bar_q = bars;                 // 1
+  uint8_t* sKV = smem + PL::kQBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NST * PL::kStageBytes);
+  uint64_t* bar_q = bars;                 // 1: Q in place (TMA landed, or TMEM rows + ones box written)
   uint64_t* kv_full = bars + 1;           // NST
-  uint64_t* kv_empty = bars + 1 + NST;    // NST
-  uint64_t* s_full = bars + 1 + 2 * NST;  // 2
-  uint64_t* p_ready = s_full + 2;         // 2
-  uint64_t* o_bar = p_ready + 2;          // 1
-  uint64_t* drain = o_bar + 1;            // 1
+  uint64_t* kv_empty = kv_full + NST;     // NST
+  uint64_t* s_full = kv_empty + NST;      // NS
+  uint64_t* p_ready = s_full + NS;        // NS
+  uint64_t* pv_done = p_ready + NS;       // NS: P V of a tile of that S buffer completed
+  uint64_t* drain = pv_done + NS;         // 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -101,13 +130,12 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   const int last_row = min(row0 + kBlockM, p.rows_per_b) - 1;
   const int64_t kend_first = key_end_rows(p.g, row0 / tok_div);
   const int64_t kend_last = key_end_rows(p.g, last_row / tok_div);
-  const int n_kv = (int)((kend_last + kBlockN - 1) / kBlockN);
+  const int n_kv = (int)((kend_last + BN - 1) / BN);
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
+    mbar_init(bar_q, Q_TMEM ? 128 : 1);
     for (int s = 0; s < NST; ++s) { mbar_init(kv_full + s, 1); mbar_init(kv_empty + s, 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(s_full + s, 1); mbar_init(p_ready + s, 128); }
-    mbar_init(o_bar, 1);
+    for (int s = 0; s < NS; ++s) { mbar_init(s_full + s, 1); mbar_init(p_ready + s, 128); mbar_init(pv_done + s, 1); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -125,12 +153,13 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   if (warp == 4) {
     // ================= TMA producer =================
     if (elect_one()) {
-      tma_prefetch_desc(&map_q);
       tma_prefetch_desc(&map_k);
       if (!V_ALIAS) tma_prefetch_desc(&map_v);
-      mbar_arrive_expect_tx(bar_q, P::kQBytes);
-      for (int i = 0; i < KB; ++i) tma_load_4d(sQ + i * kBoxBytes, &map_q, bar_q, 64 * i, h, row0, b);
-      if (KR) tma_load_4d(sQ + KB * kBoxBytes, &map_qr, bar_q, 64 * KB, h, row0, b);
+      if (!Q_TMEM) {
+        mbar_arrive_expect_tx(bar_q, PL::kQBytes);
+        for (int i = 0; i < KB; ++i) tma_load_4d(sQ + i * kBlockM * 128, &map_q, bar_q, 64 * i, h, row0, b);
+        if (KR) tma_load_4d(sQ + KB * kBlockM * 128, &map_qr, bar_q, 64 * KB, h, row0, b);
+      }
       int issued = 0;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % NST;
@@ -138,18 +167,18 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           break;
         issued = j + 1;
         if (j == p.drop_kv_tile) continue;
-        uint8_t* stage = sKV + st * P::kStageBytes;
-        mbar_arrive_expect_tx(kv_full + st, P::kStageBytes);
-        const int krow = j * kBlockN;
-        for (int i = 0; i < KB; ++i) tma_load_4d(stage + i * kBoxBytes, &map_k, kv_full + st, 64 * i, h, krow, b);
-        if (KR) tma_load_4d(stage + KB * kBoxBytes, &map_kr, kv_full + st, 0, 0, krow, b);
+        uint8_t* stage = sKV + st * PL::kStageBytes;
+        mbar_arrive_expect_tx(kv_full + st, PL::kLoadBytes);
+        const int krow = j * BN;
+        for (int i = 0; i < KB; ++i) tma_load_4d(stage + i * PL::kBox, &map_k, kv_full + st, 64 * i, h, krow, b);
+        if (KR) tma_load_4d(stage + PL::kRopeOff, &map_kr, kv_full + st, 0, 0, krow, b);
         if (!V_ALIAS)
           for (int i = 0; i < VB; ++i)
-            tma_load_4d(stage + P::kKBytes + i * kBoxBytes, &map_v, kv_full + st, 64 * i, h, krow, b);
+            tma_load_4d(stage + PL::kVOff + i * PL::kBox, &map_v, kv_full + st, 64 * i, h, krow, b);
       }
       if (*abort_flag) {
         // let the copies already issued land before the CTA exits
-        mbar_wait(bar_q, 0, &zero_flag, nullptr, 0, p.limit_ns);
+        if (!Q_TMEM) mbar_wait(bar_q, 0, &zero_flag, nullptr, 0, p.limit_ns);
         for (int j = (issued > NST ? issued - NST : 0); j < issued; ++j)
           if (j != p.drop_kv_tile) mbar_wait(kv_full + j % NST, (j / NST) & 1, &zero_flag, nullptr, 0, p.limit_ns);
       }
@@ -157,100 +186,150 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   } else if (warp == 5) {
     // ================= MMA issuer =================
     if (elect_one()) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, DV, 0, 1);
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, BN, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, PL::kNPV, 0, 1);
       const uint32_t q_base = smem_u32(sQ);
       const uint32_t kv_base = smem_u32(sKV);
       bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, 2, p.limit_ns);
       auto issue_pv = [&](int jp) -> bool {
-        const int bp = jp & 1;
-        if (!mbar_wait(p_ready + bp, (jp >> 1) & 1, abort_flag, p.status, 3, p.limit_ns)) return false;
+        const int bp = jp % NS;
+        if (!mbar_wait(p_ready + bp, (jp / NS) & 1, abort_flag, p.status, 3, p.limit_ns)) return false;
         tc_fence_after();
-        const uint32_t v_base = kv_base + (jp % NST) * P::kStageBytes + (V_ALIAS ? 0 : P::kKBytes);
+        const uint32_t v_base = kv_base + (jp % NST) * PL::kStageBytes + PL::kVOff;
 #pragma unroll
-        for (int k = 0; k < kBlockN / 16; ++k) {
-          // V tile [128 keys][64*VB] as MN-major operand: 8-key groups 1024 B apart (SBO), 64-column
-          // boxes 16 KB apart (LBO); each K step of 16 keys advances 2048 B.
-          const uint64_t vdesc = smem_desc(v_base + k * 2048, kBoxBytes, 1024, kSwizzle128B);
-          mma_ts(tmem + kTmemO, tmem + bp * 128 + k * 8, vdesc, idesc_pv, (jp > 0 || k > 0) ? 1u : 0u);
+        for (int k = 0; k < BN / 16; ++k) {
+          // V tile [BN keys][NPV] as MN-major operand: 8-key groups 1024 B apart (SBO), 64-column
+          // boxes BN*128 B apart (LBO, the ones box being the last); a K step of 16 keys is 2048 B.
+          const uint64_t vdesc = smem_desc(v_base + k * 2048, PL::kBox, 1024, kSwizzle128B);
+          mma_ts(tmem + PL::kTmemO, tmem + bp * BN + k * 8, vdesc, idesc_pv, (jp > 0 || k > 0) ? 1u : 0u);
         }
         mma_commit(kv_empty + (jp % NST));
-        mma_commit(o_bar);
+        mma_commit(pv_done + bp);
         return true;
       };
+      if (ok) tc_fence_after();
       for (int j = 0; ok && j < n_kv; ++j) {
-        const int st = j % NST, bj = j & 1;
+        const int st = j % NST, bj = j % NS;
         if (!mbar_wait(kv_full + st, (j / NST) & 1, abort_flag, p.status, 4, p.limit_ns)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t k_base = kv_base + st * P::kStageBytes;
+        // S buffer bj last held P_{j-NS}, whose P V was issued before this point (in order)
+        const uint32_t k_base = kv_base + st * PL::kStageBytes;
+        const uint32_t s_addr = tmem + bj * BN;
 #pragma unroll
         for (int k = 0; k < KB * 4; ++k) {
-          const uint32_t off = (k >> 2) * kBoxBytes + (k & 3) * 32;
-          mma_ss(tmem + bj * 128, smem_desc(q_base + off, 16, 1024, kSwizzle128B),
-                 smem_desc(k_base + off, 16, 1024, kSwizzle128B), idesc_qk, k > 0 ? 1u : 0u);
+          // 16 columns of the key tile: box k/4, 32-byte step k%4 inside the 128-byte swizzle atom
+          const uint64_t kdesc = smem_desc(k_base + (k >> 2) * PL::kBox + (k & 3) * 32, 16, 1024, kSwizzle128B);
+          if (Q_TMEM) {
+            mma_ts(s_addr, tmem + PL::kTmemQ + k * 8, kdesc, idesc_qk, k > 0 ? 1u : 0u);
+          } else {
+            const uint64_t qdesc = smem_desc(q_base + (k >> 2) * kBlockM * 128 + (k & 3) * 32, 16, 1024, kSwizzle128B);
+            mma_ss(s_addr, qdesc, kdesc, idesc_qk, k > 0 ? 1u : 0u);
+          }
         }
         if (KR) {
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const uint32_t off = KB * kBoxBytes + k * 32;
-            mma_ss(tmem + bj * 128, smem_desc(q_base + off, 16, 512, kSwizzle64B),
-                   smem_desc(k_base + off, 16, 512, kSwizzle64B), idesc_qk, 1u);
+          for (int k = 0; k < KR / 16; ++k) {
+            const uint64_t kdesc = smem_desc(k_base + PL::kRopeOff + k * 32, 16, 512, kSwizzle64B);
+            if (Q_TMEM) {
+              mma_ts(s_addr, tmem + PL::kTmemQ + KB * 32 + k * 8, kdesc, idesc_qk, 1u);
+            } else {
+              const uint64_t qdesc = smem_desc(q_base + KB * kBlockM * 128 + k * 32, 16, 512, kSwizzle64B);
+              mma_ss(s_addr, qdesc, kdesc, idesc_qk, 1u);
+            }
           }
         }
         mma_commit(s_full + bj);
-        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+        if (j >= NS - 1 && !issue_pv(j - (NS - 1))) { ok = false; break; }
       }
-      if (ok && n_kv > 0) issue_pv(n_kv - 1);
-      // every MMA of this CTA has completed before TMEM is released
+      for (int jp = (n_kv > NS - 1 ? n_kv - (NS - 1) : 0); ok && jp < n_kv; ++jp)
+        if (!issue_pv(jp)) ok = false;
+      // every MMA of this CTA has completed before TMEM is released; the softmax warps also wait
+      // on this single-phase barrier for the final O
       mma_commit(drain);
       mbar_wait(drain, 0, &zero_flag, nullptr, 0, p.limit_ns);
     }
   } else {
-    // ================= softmax + epilogue (warps 0-3, thread = query row = TMEM lane) =================
+    // ========= query rows, softmax, epilogue (warps 0-3; thread = query row = TMEM lane) =========
     const int r = threadIdx.x;                      // 0..127
     const int row = row0 + r;
     const bool row_valid = row < p.rows_per_b;
     const int64_t kend = row_valid ? key_end_rows(p.g, row / tok_div) : kend_last;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    int64_t orow;                                   // this row's index in [rows of q / out / lse]
+    if (p.dense) orow = (((int64_t)b * p.nq + row) * p.heads + h);
+    else orow = (int64_t)b * p.rows_per_b + row;
+
+    if (Q_TMEM) {
+      if (ONES) {
+        // 16 columns of ones after V in every stage (bf16 1.0 everywhere in the box, so the swizzle
+        // does not matter); made visible to the tensor cores' async proxy before bar_q is released
+        constexpr int kWords = NST * PL::kBox / 16;
+#pragma unroll 4
+        for (int i = r; i < kWords; i += 128) {
+          const int st = i / (PL::kBox / 16), w = i % (PL::kBox / 16);
+          reinterpret_cast<uint4*>(sKV + st * PL::kStageBytes + PL::kOnesOff)[w] =
+              make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+        }
+        fence_proxy_async_smem();
+      }
+      // the Q row as 32-bit words (bf16 pairs) into TMEM columns [kTmemQ, kTmemQ + DQK/2): exactly the
+      // A-operand layout of a 128-row tcgen05.mma (row = lane, K pairs along columns)
+      const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.q) + orow * DQK);
+#pragma unroll
+      for (int c0 = 0; c0 < DQK / 2; c0 += 8) {
+        uint32_t w[8];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const uint4 v = row_valid ? src[c0 / 4 + q] : make_uint4(0, 0, 0, 0);
+          w[4 * q + 0] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+        }
+        tmem_st8(tmem + lane_base + PL::kTmemQ + c0, w);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_q);
+    }
+
     float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = true;
-    // Wait until P_{k} V_{k} has completed (phase k of o_bar).  Only called from tile j = k + 1,
-    // where o_bar is at most one phase away from phase k: s_full[j] completing implies that
-    // P_{j-2} V_{j-2} completed (it was issued before S_j), and P_j V_j cannot start before this
-    // thread releases P_j, so a parity wait is unambiguous.  Warp-uniform (__all_sync) because the
-    // TMEM loads/stores that follow are warp-collective.
+    // Wait until P_{j-1} V_{j-1} has completed: phase (j-1)/NS of pv_done[(j-1) % NS].  Called from tile
+    // j, where that barrier is at most one phase away: s_full[j] completing implies that
+    // P_{j-1-NS} V_{j-1-NS} completed (issued before S_j), and P_{j-1+NS} V_{j-1+NS} cannot start
+    // before this thread releases its P, so a parity wait is unambiguous.  Warp-uniform (__all_sync)
+    // because the TMEM loads/stores that follow are warp-collective.
     auto wait_pv = [&](int k) -> bool {
-      const bool got = mbar_wait(o_bar, k & 1, abort_flag, p.status, 5, p.limit_ns);
+      const bool got = mbar_wait(pv_done + k % NS, (k / NS) & 1, abort_flag, p.status, 5, p.limit_ns);
       return __all_sync(0xffffffffu, got);
     };
+    const float sc = p.scale_log2;
     for (int j = 0; j < n_kv; ++j) {
-      const int bj = j & 1;
-      const bool got = mbar_wait(s_full + bj, (j >> 1) & 1, abort_flag, p.status, 6, p.limit_ns);
+      const int bj = j % NS;
+      const bool got = mbar_wait(s_full + bj, (j / NS) & 1, abort_flag, p.status, 6, p.limit_ns);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      // S row of this thread (raw scores): four 32-column TMEM loads, one wait
-      uint32_t sr[kBlockN];
+      // S row of this thread (raw scores): BN/32 TMEM loads, one wait
+      float sr[BN];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(tmem + lane_base + bj * 128 + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
+      for (int c = 0; c < BN / 32; ++c)
+        tmem_ld32(tmem + lane_base + bj * BN + c * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
       tmem_ld_wait();
-      const int64_t key0 = (int64_t)j * kBlockN;
-      if (key0 + kBlockN > kend_first) {
+      const int64_t key0 = (int64_t)j * BN;
+      if (key0 + BN > kend_first) {
 #pragma unroll
-        for (int i = 0; i < kBlockN; ++i)
-          if (key0 + i >= kend) sr[i] = __float_as_uint(-INFINITY);
+        for (int i = 0; i < BN; ++i)
+          if (key0 + i >= kend) sr[i] = -INFINITY;
       }
-      // row max as a tree of 8 independent chains (the scale is positive, so it is applied after)
+      // row max: 8 chains of 3-input max, then a tree (the scale is positive, applied after)
+      static_assert(BN % 16 == 0 && BN >= 32, "max chains");
       float mx[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(sr[i]);
+      for (int q = 0; q < 8; ++q) mx[q] = fmaxf(sr[q], sr[8 + q]);                 // keys 0..15
 #pragma unroll
-      for (int i = 8; i < kBlockN; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(sr[i]));
+      for (int i = 16; i < BN; i += 16)                                              // keys i..i+15
 #pragma unroll
-      for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-        for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
-      const float m_new = fmaxf(m_ref, mx[0] * p.scale_log2);
+        for (int q = 0; q < 8; ++q) mx[q] = fmax3(mx[q], sr[i + q], sr[i + 8 + q]);
+      const float m_tile = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmaxf(fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float m_new = fmaxf(m_ref, m_tile * sc);
       const bool need = m_new > m_ref + kRescaleThreshold;
       if (__any_sync(0xffffffffu, need)) {
         const float alpha = fast_exp2(m_ref - m_new);   // 0 on the first tile
@@ -260,58 +339,69 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           uint32_t o[32];
 #pragma unroll
           for (int c = 0; c < DV / 32; ++c) {
-            tmem_ld32(tmem + lane_base + kTmemO + c * 32, o);
+            tmem_ld32(tmem + lane_base + PL::kTmemO + c * 32, o);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tmem + lane_base + kTmemO + c * 32, o);
+            tmem_st32(tmem + lane_base + PL::kTmemO + c * 32, o);
+          }
+          if (ONES) {                                   // the row-sum column rescales with O
+            tmem_ld16(tmem + lane_base + PL::kTmemO + DV, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st16(tmem + lane_base + PL::kTmemO + DV, *reinterpret_cast<uint32_t(*)[16]>(o));
           }
         }
         l_sum *= alpha;
         m_ref = m_new;
       }
-      // p = 2^(s * scale*log2(e) - m) (one FFMA + one MUFU.EX2 per score), row sum in 8 chains,
-      // P packed to bf16 pairs over the first 64 columns of this S buffer
+      // p = 2^(s * scale*log2(e) - m): one packed FMA per pair of scores, then MUFU.EX2; P packed to
+      // bf16 pairs over the first BN/2 columns of this S buffer (row sums: the ones columns of V, or
+      // 4 packed chains)
       const float neg_m = -m_ref;
       float ls[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) ls[i] = 0.f;
-      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < BN / 16; ++c) {
+        uint32_t pk[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c * 64 + 2 * i]), p.scale_log2, neg_m));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c * 64 + 2 * i + 1]), p.scale_log2, neg_m));
-          ls[(2 * i) & 7] += p0;
-          ls[(2 * i + 1) & 7] += p1;
+        for (int i = 0; i < 8; ++i) {
+          float x0, x1;
+          ffma2(x0, x1, sr[c * 16 + 2 * i], sr[c * 16 + 2 * i + 1], sc, sc, neg_m, neg_m);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          if (!ONES) fadd2(ls[(2 * i) & 7], ls[(2 * i + 1) & 7], p0, p1);
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(tmem + lane_base + bj * 128 + c * 32, pk);
+        tmem_st8(tmem + lane_base + bj * BN + c * 8, pk);
       }
-#pragma unroll
-      for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-        for (int i = 0; i < w; ++i) ls[i] += ls[i + w];
-      l_sum += ls[0];
+      if (!ONES) {
+        fadd2(ls[0], ls[1], ls[4], ls[5]);
+        fadd2(ls[2], ls[3], ls[6], ls[7]);
+        fadd2(ls[0], ls[1], ls[2], ls[3]);
+        l_sum += ls[0] + ls[1];
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_ready + bj);
     }
-    // `drain` is committed once, after the last P*V, so its single phase marks O complete
     bool fin = ok && mbar_wait(drain, 0, abort_flag, p.status, 7, p.limit_ns);
     fin = __all_sync(0xffffffffu, fin && !*abort_flag);
     if (fin) {
       tc_fence_after();
-      const float inv_l = 1.f / l_sum;
-      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
-      int64_t orow;
-      if (p.dense) orow = (((int64_t)b * p.nq + row) * p.heads + h);
-      else orow = (int64_t)b * p.rows_per_b + row;
       uint32_t o[32];
+      float l_row = l_sum;
+      if (ONES) {
+        tmem_ld16(tmem + lane_base + PL::kTmemO + DV, o);
+        tmem_ld_wait();
+        l_row = __uint_as_float(o[0]);
+      }
+      const float inv_l = 1.f / l_row;
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
 #pragma unroll
       for (int c = 0; c < DV / 32; ++c) {
-        tmem_ld32(tmem + lane_base + kTmemO + c * 32, o);
+        tmem_ld32(tmem + lane_base + PL::kTmemO + c * 32, o);
         tmem_ld_wait();
         if (row_valid) {
           uint4* dst = reinterpret_cast<uint4*>(out + orow * DV + c * 32);
@@ -326,7 +416,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           }
         }
       }
-      if (row_valid && p.lse) p.lse[orow] = (m_ref + __log2f(l_sum)) * 0.69314718055994530942f;
+      if (row_valid && p.lse) p.lse[orow] = (m_ref + __log2f(l_row)) * 0.69314718055994530942f;
     }
   }
   tc_fence_before();
@@ -337,22 +427,25 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   }
 }
 
-template <int KB, int KR, int VB, bool V_ALIAS>
-std::atomic<uint64_t>& attr_done() {
-  static std::atomic<uint64_t> mask{0};
-  return mask;
-}
-
-template <int KB, int KR, int VB, bool V_ALIAS>
+template <int KB, int KR, int VB, bool V_ALIAS, int BN, int NS, bool Q_TMEM, bool ONES>
 cudaError_t launch_attention(const TmaMaps5& m, const AttnParams& p, int n_tiles, cudaStream_t st) {
-  using PL = Plan<KB, KR, VB, V_ALIAS>;
-  auto kern = attention_kernel<KB, KR, VB, V_ALIAS>;
-  cudaError_t attr_err = ensure_smem_attr((const void*)kern, PL::kSmemBytes, attr_done<KB, KR, VB, V_ALIAS>());
+  using PL = Plan<KB, KR, VB, V_ALIAS, BN, NS, Q_TMEM, ONES>;
+  auto kern = attention_kernel<KB, KR, VB, V_ALIAS, BN, NS, Q_TMEM, ONES>;
+  static std::atomic<uint64_t> done{0};
+  cudaError_t attr_err = ensure_smem_attr((const void*)kern, PL::kSmemBytes, done);
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<n_tiles, kThreads, PL::kSmemBytes, st>>>(m.q, m.qr, m.k, m.kr, m.v, p);
   count_launches(1);
   return cudaGetLastError();
 }
+
+// Instances (measured on B200; the softmax warps bound these kernels, the MMA side alone reaches the
+// full tensor rate in every one of them):
+//   latent d_c = 192 / 256: Q in shared memory, 128-key tiles, two S buffers (fastest per key);
+//   latent d_c = 64 / 128 and the dense layer: Q in TMEM, 128-key tiles, two S buffers.
+// The three-buffer / 64-key / ones-column variant of the template is correct but slower at these
+// shapes (its per-tile fixed costs outweigh the shorter dependency chain).
+constexpr int kLatentBN = 128;
 
 }  // namespace
 
@@ -380,19 +473,21 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
                                 cudaStream_t st) {
   const int H = cfg.n_heads, dqk = cfg.d_c + cfg.d_rope;
   const int64_t rows = nq * H;
+  const int kv_box_rows = kLatentBN;
   TmaMaps5 m{};
   cudaError_t e;
-  // q_abs [B, Nq*H, d_qk] viewed as 4D {d_qk, 1, Nq*H, B}
+  // q_abs [B, Nq*H, d_qk] viewed as 4D {d_qk, 1, Nq*H, B} (only read by TMA when Q stays in smem)
   if ((e = make_map_4d(&m.q, q_abs, dqk, 1, rows, batch, (int64_t)dqk * 2, (int64_t)dqk * 2,
                        rows * dqk * 2, 64, 1, kBlockM, 128)) != cudaSuccess) return e;
   if ((e = make_map_4d(&m.qr, q_abs, dqk, 1, rows, batch, (int64_t)dqk * 2, (int64_t)dqk * 2,
                        rows * dqk * 2, 32, 1, kBlockM, 64)) != cudaSuccess) return e;
   if ((e = make_map_4d(&m.k, c, cfg.d_c, 1, valid_rows, batch, (int64_t)cfg.d_c * 2, (int64_t)cfg.d_c * 2,
-                       cap * cfg.d_c * 2, 64, 1, kBlockN, 128)) != cudaSuccess) return e;
-  if ((e = make_map_4d(&m.kr, k_r, 32, 1, valid_rows, batch, 64, 64, cap * 64, 32, 1, kBlockN, 64)) != cudaSuccess)
+                       cap * cfg.d_c * 2, 64, 1, kv_box_rows, 128)) != cudaSuccess) return e;
+  if ((e = make_map_4d(&m.kr, k_r, 32, 1, valid_rows, batch, 64, 64, cap * 64, 32, 1, kv_box_rows, 64)) != cudaSuccess)
     return e;
   m.v = m.k;
   AttnParams p{};
+  p.q = q_abs;
   p.rows_per_b = (int)rows;
   p.tiles_per_group = (int)((rows + kBlockM - 1) / kBlockM);
   p.heads = H;
@@ -407,10 +502,10 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
   p.drop_kv_tile = take_drop_kv_tile();
   const int n_tiles = batch * p.tiles_per_group;
   switch (cfg.d_c) {
-    case 64: return launch_attention<1, 32, 1, true>(m, p, n_tiles, st);
-    case 128: return launch_attention<2, 32, 2, true>(m, p, n_tiles, st);
-    case 192: return launch_attention<3, 32, 3, true>(m, p, n_tiles, st);
-    default: return launch_attention<4, 32, 4, true>(m, p, n_tiles, st);
+    case 64: return launch_attention<1, 32, 1, true, kLatentBN, 2, true, false>(m, p, n_tiles, st);
+    case 128: return launch_attention<2, 32, 2, true, kLatentBN, 2, true, false>(m, p, n_tiles, st);
+    case 192: return launch_attention<3, 32, 3, true, kLatentBN, 2, false, false>(m, p, n_tiles, st);
+    default: return launch_attention<4, 32, 4, true, kLatentBN, 2, false, false>(m, p, n_tiles, st);
   }
 }
 
@@ -419,17 +514,19 @@ cudaError_t tc_dense_mha(const vmla_config& cfg, int batch, int64_t nq, const vo
                          float scale, void* out, float* lse, int* status, cudaStream_t st) {
   const int H = cfg.n_heads;
   const int D = 128;
+  constexpr int kBN = 128;
   TmaMaps5 m{};
   cudaError_t e;
   if ((e = make_map_4d(&m.q, q, D, H, nq, batch, D * 2, (int64_t)H * D * 2, nq * H * D * 2, 64, 1, kBlockM,
                        128)) != cudaSuccess) return e;
   m.qr = m.q;
   if ((e = make_map_4d(&m.k, k, D, H, valid_rows, batch, D * 2, (int64_t)H * D * 2, cap * H * D * 2, 64, 1,
-                       kBlockN, 128)) != cudaSuccess) return e;
+                       kBN, 128)) != cudaSuccess) return e;
   m.kr = m.k;
   if ((e = make_map_4d(&m.v, v, D, H, valid_rows, batch, D * 2, (int64_t)H * D * 2, cap * H * D * 2, 64, 1,
-                       kBlockN, 128)) != cudaSuccess) return e;
+                       kBN, 128)) != cudaSuccess) return e;
   AttnParams p{};
+  p.q = q;
   p.rows_per_b = (int)nq;
   p.tiles_per_group = (int)((nq + kBlockM - 1) / kBlockM);
   p.heads = H;
@@ -443,7 +540,7 @@ cudaError_t tc_dense_mha(const vmla_config& cfg, int batch, int64_t nq, const vo
   p.limit_ns = wait_limit_ns();
   p.drop_kv_tile = -1;
   const int n_tiles = batch * H * p.tiles_per_group;
-  return launch_attention<2, 0, 2, false>(m, p, n_tiles, st);
+  return launch_attention<2, 0, 2, false, kBN, 2, true, false>(m, p, n_tiles, st);
 }
 
 }  // namespace vmla
