@@ -7,9 +7,11 @@
 //   value_up         o_h = W^V_up,h o~_h per head (Method item 2);
 //   dense_append     the dense comparison layer's per-head K and V projection (RoPE on each head's
 //                    last d_rope key columns) into the dense ring.
-// One CTA computes one 128-row x BN tile: warp 0 streams A/B k-tiles with TMA into a 4-deep ring,
-// warp 1 owns TMEM and issues tcgen05.mma (K = 16 per instruction, fp32 accumulation), warps 2-5 read
-// the accumulator rows back (one thread per row) and run the epilogue.
+// Persistent kernels: one CTA per SM loops over 128-row x BN output tiles.  Warp 0 streams A/B
+// k-tiles with TMA into a shared-memory ring, warp 1 owns TMEM and issues tcgen05.mma (K = 16 per
+// instruction, fp32 accumulation) into one of two TMEM accumulators, and warps 2-5 read the other
+// accumulator back (one thread per row) and run the epilogue, so a tile's epilogue overlaps the next
+// tile's loads and MMAs.
 #include <cuda.h>
 
 #include <atomic>
@@ -33,9 +35,10 @@ struct GemmShape {
   int64_t M;          // rows of A (all batch elements)
   int N;              // output columns of this GEMM (per head)
   int K;              // reduction length
-  int a_head;         // head coordinate of A's map (0 or blockIdx.z)
+  int a_head;         // whether A's map has a head coordinate (per-head A rows)
   uint64_t limit_ns;
   int* status;
+  int heads;          // independent GEMMs (heads) sharing the shapes; set by the launcher
 };
 
 __device__ __forceinline__ void store32(bf16* dst, const float* v) {
@@ -51,21 +54,75 @@ __device__ __forceinline__ void store32(bf16* dst, const float* v) {
   }
 }
 
-__device__ __forceinline__ void rope32(const RopeTable& rt, int pair0, int64_t f, int64_t i, int64_t j,
-                                       float* v) {
+// 3D-RoPE of the epilogues through a per-CTA table: cos/sin of every (rotary pair, position along its
+// axis) that the call can meet -- the call's frames, every row, every column -- computed once per CTA
+// in shared memory (angle reduced in double precision, then sincosf).  Pair p's entries start at
+// off[p]; frame positions are stored relative to base_f.  n_entries == 0 (table too large) falls back
+// to computing each rotation directly.
+constexpr int kRopeTabEntries = 2048;
+
+struct RopeLookup {
+  RopeTable rt;
+  int off[kMaxRopePairs];
+  int64_t base_f;
+  int n_entries;
+  __device__ void rotate32(const float2* tab, int pair0, int64_t f, int64_t i, int64_t j, float* v) const {
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    float a, b;
-    rope_rotate_f32(rt, pair0 + q, f, i, j, v[2 * q], v[2 * q + 1], &a, &b);
-    v[2 * q] = a;
-    v[2 * q + 1] = b;
+    for (int q = 0; q < 16; ++q) {
+      const int p = pair0 + q;
+      float a, b;
+      if (n_entries) {
+        const int ax = rt.axis[p];
+        const int64_t pos = ax == 0 ? f - base_f : (ax == 1 ? i : j);
+        const float2 cs = tab[off[p] + pos];
+        a = v[2 * q] * cs.x - v[2 * q + 1] * cs.y;
+        b = v[2 * q] * cs.y + v[2 * q + 1] * cs.x;
+      } else {
+        rope_rotate_f32(rt, p, f, i, j, v[2 * q], v[2 * q + 1], &a, &b);
+      }
+      v[2 * q] = a;
+      v[2 * q + 1] = b;
+    }
   }
+
+  // fill the table (all threads of the CTA), then __syncthreads()
+  __device__ void build(float2* smem_tab) const {
+    const double two_pi = 6.283185307179586476925286766559;
+    const double inv_two_pi = 0.15915494309189533576888376337251;
+    for (int e = threadIdx.x; e < n_entries; e += blockDim.x) {
+      int p = 0;
+      while (p + 1 < rt.n_pairs && off[p + 1] <= e) ++p;
+      const int64_t v = e - off[p];
+      const double pos = (double)(rt.axis[p] == 0 ? base_f + v : v);
+      double ang = pos * rt.inv_freq[p];
+      ang = fma(-two_pi, rint(ang * inv_two_pi), ang);
+      float sn, cs;
+      sincosf((float)ang, &sn, &cs);
+      smem_tab[e] = make_float2(cs, sn);
+    }
+  }
+};
+
+// Host: table layout for a call whose tokens span `frames` frames starting at g.first_frame.
+RopeLookup make_rope_lookup(const RopeTable& rt, const FrameGeom& g, int frames) {
+  RopeLookup L{};
+  L.rt = rt;
+  L.base_f = g.first_frame;
+  const int extent[3] = {frames, g.tokens_per_frame / g.grid_w, g.grid_w};
+  int total = 0;
+  for (int p = 0; p < rt.n_pairs; ++p) {
+    L.off[p] = total;
+    total += extent[rt.axis[p]];
+  }
+  L.n_entries = total <= kRopeTabEntries ? total : 0;
+  return L;
 }
 
 // ---- epilogues: called per (row m, 32-column chunk starting at col0) with the fp32 values ----
 struct EpiCompress {
-  bf16* c; bf16* k_r; int d_c, d_rope; int64_t ntok, cap; FrameGeom g; RopeTable rt;
-  __device__ void operator()(int, int64_t m, int col0, float* v) const {
+  static constexpr bool kRope = true;
+  bf16* c; bf16* k_r; int d_c, d_rope; int64_t ntok, cap; FrameGeom g; RopeLookup rope;
+  __device__ void operator()(const float2* tab, int, int64_t m, int col0, float* v) const {
     const int64_t b = m / ntok, tok = m % ntok;
     const int64_t row = b * cap + ring_row(g, tok);
     if (col0 < d_c) {
@@ -73,20 +130,21 @@ struct EpiCompress {
     } else {
       const int64_t f = g.first_frame + tok / g.tokens_per_frame;
       const int64_t r = tok % g.tokens_per_frame;
-      rope32(rt, (col0 - d_c) / 2, f, r / g.grid_w, r % g.grid_w, v);
+      rope.rotate32(tab, (col0 - d_c) / 2, f, r / g.grid_w, r % g.grid_w, v);
       store32(k_r + row * d_rope + (col0 - d_c), v);
     }
   }
-  __device__ void finish(int, int64_t) const {}
+  __device__ void finish(const float2*, int, int64_t) const {}
 };
 
 struct EpiAbsorb {
-  bf16* q_abs; const bf16* q_rope; int heads, d_c, d_rope; int64_t nq; FrameGeom g; RopeTable rt;
-  __device__ void operator()(int h, int64_t m, int col0, float* v) const {
+  static constexpr bool kRope = true;
+  bf16* q_abs; const bf16* q_rope; int heads, d_c, d_rope; int64_t nq; FrameGeom g; RopeLookup rope;
+  __device__ void operator()(const float2* tab, int h, int64_t m, int col0, float* v) const {
     store32(q_abs + (m * heads + h) * (d_c + d_rope) + col0, v);
   }
   // RoPE3D(q^rope) of row m, head h -> q_abs[m, h, d_c : d_c + d_rope]
-  __device__ void finish(int h, int64_t m) const {
+  __device__ void finish(const float2* tab, int h, int64_t m) const {
     const int64_t tok = m % nq;
     const int64_t f = g.first_frame + tok / g.tokens_per_frame;
     const int64_t r = tok % g.tokens_per_frame;
@@ -101,23 +159,26 @@ struct EpiAbsorb {
 #pragma unroll
         for (int t = 0; t < 8; ++t) v[8 * q + t] = __bfloat162float(e[t]);
       }
-      rope32(rt, c0 / 2, f, r / g.grid_w, r % g.grid_w, v);
+      rope.rotate32(tab, c0 / 2, f, r / g.grid_w, r % g.grid_w, v);
       store32(q_abs + (m * heads + h) * (d_c + d_rope) + d_c + c0, v);
     }
   }
 };
 
 struct EpiValueUp {
+  static constexpr bool kRope = false;
+  RopeLookup rope;   // unused
   bf16* out; int heads, d_v;
-  __device__ void operator()(int h, int64_t m, int col0, float* v) const {
+  __device__ void operator()(const float2* tab, int h, int64_t m, int col0, float* v) const {
     store32(out + (m * heads + h) * d_v + col0, v);
   }
-  __device__ void finish(int, int64_t) const {}
+  __device__ void finish(const float2*, int, int64_t) const {}
 };
 
 struct EpiDense {
-  bf16* k; bf16* v; int heads, d_nope, d_h, d_v; int64_t ntok, cap; FrameGeom g; RopeTable rt;
-  __device__ void operator()(int, int64_t m, int col0, float* x) const {
+  static constexpr bool kRope = true;
+  bf16* k; bf16* v; int heads, d_nope, d_h, d_v; int64_t ntok, cap; FrameGeom g; RopeLookup rope;
+  __device__ void operator()(const float2* tab, int, int64_t m, int col0, float* x) const {
     const int64_t b = m / ntok, tok = m % ntok;
     const int64_t row = b * cap + ring_row(g, tok);
     if (col0 < heads * d_h) {
@@ -125,7 +186,7 @@ struct EpiDense {
       if (cc >= d_nope) {
         const int64_t f = g.first_frame + tok / g.tokens_per_frame;
         const int64_t r = tok % g.tokens_per_frame;
-        rope32(rt, (cc - d_nope) / 2, f, r / g.grid_w, r % g.grid_w, x);
+        rope.rotate32(tab, (cc - d_nope) / 2, f, r / g.grid_w, r % g.grid_w, x);
       }
       store32(k + (row * heads + hh) * d_h + cc, x);
     } else {
@@ -133,45 +194,66 @@ struct EpiDense {
       store32(v + (row * heads + cv / d_v) * d_v + cv % d_v, x);
     }
   }
-  __device__ void finish(int, int64_t) const {}
+  __device__ void finish(const float2*, int, int64_t) const {}
 };
 
-template <int BN, bool B_MN_MAJOR, int STAGES>
+template <int BN, bool B_MN_MAJOR>
 struct GemmPlan {
-  static constexpr int kStages = STAGES;
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 256 + 1024;
-  static constexpr uint32_t kTmemCols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+  static constexpr int kTabBytes = kRopeTabEntries * 8;   // RoPE table (epilogues that rotate)
+  static constexpr int kFit = (232448 - 1024 - 256 - kTabBytes) / kStageBytes;
+  static constexpr int kStages = kFit >= 6 ? 6 : kFit;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 256 + kTabBytes + 1024;
+  // one fp32 accumulator of BN columns, double-buffered in TMEM
+  static constexpr uint32_t kAccCols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+  static constexpr uint32_t kTmemCols = 2 * kAccCols;
   static_assert(BN % 32 == 0 && BN <= 256, "BN");
   static_assert(!B_MN_MAJOR || BN % 64 == 0, "MN-major B is loaded in 64-column boxes");
+  static_assert(kStages >= 2, "shared memory too small for two stages");
 };
 
-template <int BN, bool B_MN_MAJOR, int STAGES, class Epi>
+// Persistent tile loop: tile t -> (head z, column tile nt, row tile mt) with mt fastest (consecutive
+// CTAs share the weight tile); CTA c takes tiles c, c + grid, c + 2*grid, ...
+struct TileCoord { int mt, nt, z; };
+__device__ __forceinline__ TileCoord tile_coord(int t, int n_m, int n_n) {
+  TileCoord c;
+  c.z = t / (n_m * n_n);
+  const int rem = t - c.z * n_m * n_n;
+  c.nt = rem / n_m;
+  c.mt = rem - c.nt * n_m;
+  return c;
+}
+
+template <int BN, bool B_MN_MAJOR, class Epi>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-            const GemmShape sh, Epi epi) {
-  using PL = GemmPlan<BN, B_MN_MAJOR, STAGES>;
-  constexpr int kStages = STAGES;
+            const GemmShape sh, const Epi epi) {
+  using PL = GemmPlan<BN, B_MN_MAJOR>;
+  constexpr int kStages = PL::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * PL::kStageBytes);
-  uint64_t* full = bars;                 // kStages
-  uint64_t* empty = bars + kStages;      // kStages
-  uint64_t* acc_full = bars + 2 * kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* full = bars;                  // kStages
+  uint64_t* empty = full + kStages;       // kStages
+  uint64_t* acc_full = empty + kStages;   // 2: accumulator buffer ready for the epilogue
+  uint64_t* acc_empty = acc_full + 2;     // 2: accumulator buffer read back by the epilogue
+  uint64_t* drain = acc_empty + 2;        // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float2* rope_tab = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(bars) + 256);
 
   const int warp = threadIdx.x / 32;
-  const int64_t m0 = (int64_t)blockIdx.x * kBM;
-  const int n0 = blockIdx.y * BN;
-  const int head = blockIdx.z;
   const int nk = (sh.K + kBK - 1) / kBK;
+  const int n_m = (int)((sh.M + kBM - 1) / kBM);
+  const int n_n = (sh.N + BN - 1) / BN;
+  const int n_tiles = n_m * n_n * sh.heads;
   int zero_flag = 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); }
-    mbar_init(acc_full, 1);
+    for (int s = 0; s < 2; ++s) { mbar_init(acc_full + s, 1); mbar_init(acc_empty + s, 128); }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -179,84 +261,111 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
     tmem_alloc(tmem_slot, PL::kTmemCols);
     tmem_relinquish();
   }
+  if constexpr (Epi::kRope) epi.rope.build(rope_tab);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
+    // ================= TMA producer (k-iterations counted across tiles) =================
     if (elect_one()) {
       tma_prefetch_desc(&map_a);
       tma_prefetch_desc(&map_b);
-      int issued = 0;
-      for (int kt = 0; kt < nk; ++kt) {
-        const int st = kt % kStages;
-        if (kt >= kStages &&
-            !mbar_wait(empty + st, ((kt / kStages) - 1) & 1, abort_flag, sh.status, 11, sh.limit_ns))
-          break;
-        uint8_t* sa = smem + st * PL::kStageBytes;
-        uint8_t* sb = sa + kABytes;
-        mbar_arrive_expect_tx(full + st, PL::kStageBytes);
-        tma_load_4d(sa, &map_a, full + st, kt * kBK, sh.a_head ? head : 0, (int)m0, 0);
-        if (B_MN_MAJOR) {
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+        const TileCoord tc = tile_coord(t, n_m, n_n);
+        for (int kt = 0; kt < nk; ++kt, ++it) {
+          const int st = it % kStages;
+          if (it >= kStages &&
+              !mbar_wait(empty + st, ((it / kStages) - 1) & 1, abort_flag, sh.status, 11, sh.limit_ns)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + st * PL::kStageBytes;
+          uint8_t* sb = sa + kABytes;
+          mbar_arrive_expect_tx(full + st, PL::kStageBytes);
+          tma_load_4d(sa, &map_a, full + st, kt * kBK, sh.a_head ? tc.z : 0, tc.mt * kBM, 0);
+          if (B_MN_MAJOR) {
 #pragma unroll
-          for (int i = 0; i < BN / 64; ++i)
-            tma_load_4d(sb + i * (kBK * 128), &map_b, full + st, n0 + 64 * i, kt * kBK, head, 0);
-        } else {
-          tma_load_4d(sb, &map_b, full + st, kt * kBK, n0, head, 0);
+            for (int i = 0; i < BN / 64; ++i)
+              tma_load_4d(sb + i * (kBK * 128), &map_b, full + st, tc.nt * BN + 64 * i, kt * kBK, tc.z, 0);
+          } else {
+            tma_load_4d(sb, &map_b, full + st, kt * kBK, tc.nt * BN, tc.z, 0);
+          }
         }
-        issued = kt + 1;
       }
-      if (*abort_flag)
-        for (int kt = (issued > kStages ? issued - kStages : 0); kt < issued; ++kt)
-          mbar_wait(full + kt % kStages, (kt / kStages) & 1, &zero_flag, nullptr, 0, sh.limit_ns);
+      if (!ok) {
+        // let the copies already issued land before the CTA exits
+        for (int j = (it > kStages ? it - kStages : 0); j < it; ++j)
+          mbar_wait(full + j % kStages, (j / kStages) & 1, &zero_flag, nullptr, 0, sh.limit_ns);
+      }
     }
   } else if (warp == 1) {
+    // ================= MMA issuer =================
     if (elect_one()) {
       constexpr uint32_t idesc = idesc_bf16_f32(kBM, BN, 0, B_MN_MAJOR ? 1 : 0);
+      int it = 0, li = 0;
       bool ok = true;
-      for (int kt = 0; kt < nk; ++kt) {
-        const int st = kt % kStages;
-        if (!mbar_wait(full + st, (kt / kStages) & 1, abort_flag, sh.status, 12, sh.limit_ns)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t a = smem_u32(smem + st * PL::kStageBytes);
-        const uint32_t b = a + kABytes;
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          const uint64_t ad = smem_desc(a + kk * 32, 16, 1024, kSwizzle128B);
-          const uint64_t bd = B_MN_MAJOR ? smem_desc(b + kk * 2048, kBK * 128, 1024, kSwizzle128B)
-                                         : smem_desc(b + kk * 32, 16, 1024, kSwizzle128B);
-          mma_ss(tmem, ad, bd, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++li) {
+        const int ab = li & 1;
+        if (li >= 2 && !mbar_wait(acc_empty + ab, ((li >> 1) - 1) & 1, abort_flag, sh.status, 14, sh.limit_ns)) {
+          ok = false;
+          break;
         }
-        mma_commit(empty + st);
+        tc_fence_after();
+        const uint32_t acc = tmem + ab * PL::kAccCols;
+        for (int kt = 0; kt < nk; ++kt, ++it) {
+          const int st = it % kStages;
+          if (!mbar_wait(full + st, (it / kStages) & 1, abort_flag, sh.status, 12, sh.limit_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + st * PL::kStageBytes);
+          const uint32_t b = a + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = smem_desc(a + kk * 32, 16, 1024, kSwizzle128B);
+            const uint64_t bd = B_MN_MAJOR ? smem_desc(b + kk * 2048, kBK * 128, 1024, kSwizzle128B)
+                                           : smem_desc(b + kk * 32, 16, 1024, kSwizzle128B);
+            mma_ss(acc, ad, bd, idesc, (kt > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(empty + st);
+        }
+        if (ok) mma_commit(acc_full + ab);
       }
-      mma_commit(acc_full);
-      (void)ok;
       // every MMA of this CTA has completed before TMEM is released
-      mbar_wait(acc_full, 0, &zero_flag, nullptr, 0, sh.limit_ns);
+      mma_commit(drain);
+      mbar_wait(drain, 0, &zero_flag, nullptr, 0, sh.limit_ns);
     }
   } else {
-    // epilogue: warps 2..5, TMEM lane quadrant = warp % 4
+    // ================= epilogue: warps 2..5, TMEM lane quadrant = warp % 4 =================
     const int quad = warp & 3;
     const int r = quad * 32 + (threadIdx.x & 31);
-    const int64_t m = m0 + r;
-    const bool got = mbar_wait(acc_full, 0, abort_flag, sh.status, 13, sh.limit_ns);
-    if (__all_sync(0xffffffffu, got)) {     // the TMEM loads below are warp-collective
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    int li = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++li) {
+      const TileCoord tc = tile_coord(t, n_m, n_n);
+      const int ab = li & 1;
+      const bool got = mbar_wait(acc_full + ab, (li >> 1) & 1, abort_flag, sh.status, 13, sh.limit_ns);
+      if (!__all_sync(0xffffffffu, got)) break;      // the TMEM loads below are warp-collective
       tc_fence_after();
-      const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+      const int64_t m = (int64_t)tc.mt * kBM + r;
+      const int n0 = tc.nt * BN;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t raw[32];
-        tmem_ld32(tmem + lane_base + c0, raw);
+        tmem_ld32(tmem + lane_base + ab * PL::kAccCols + c0, raw);
         tmem_ld_wait();
         if (m < sh.M && n0 + c0 < sh.N) {
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
-          epi(head, m, n0 + c0, v);
+          epi(rope_tab, tc.z, m, n0 + c0, v);
         }
       }
-      if (m < sh.M && blockIdx.y == 0) epi.finish(head, m);
+      tc_fence_before();
+      mbar_arrive(acc_empty + ab);
+      if (m < sh.M && tc.nt == 0) epi.finish(rope_tab, tc.z, m);
     }
   }
   tc_fence_before();
@@ -267,27 +376,34 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
   }
 }
 
-template <int BN, bool B_MN_MAJOR, int STAGES, class Epi>
-cudaError_t launch_gemm_st(const CUtensorMap& a, const CUtensorMap& b, const GemmShape& sh, int heads,
-                           const Epi& epi, cudaStream_t st) {
-  using PL = GemmPlan<BN, B_MN_MAJOR, STAGES>;
-  auto kern = gemm_kernel<BN, B_MN_MAJOR, STAGES, Epi>;
-  static std::atomic<uint64_t> done{0};
-  cudaError_t attr_err = ensure_smem_attr((const void*)kern, PL::kSmemBytes, done);
-  if (attr_err != cudaSuccess) return attr_err;
-  dim3 grid((unsigned)((sh.M + kBM - 1) / kBM), (unsigned)((sh.N + BN - 1) / BN), (unsigned)heads);
-  kern<<<grid, kThreads, PL::kSmemBytes, st>>>(a, b, sh, epi);
-  count_launches(1);
-  return cudaGetLastError();
+int num_sms() {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cached[dev] = v;
+  }
+  return cached[dev];
 }
 
-// Short reductions (K <= 2 k-tiles per stage ring) use a 2-deep ring so that several CTAs share an SM
-// and one CTA's epilogue overlaps another's loads; long ones (the D = 1536 projections) a 4-deep ring.
+// One CTA per SM (TMEM holds two accumulators), each looping over its share of the tiles.
 template <int BN, bool B_MN_MAJOR, class Epi>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmShape& sh, int heads,
                         const Epi& epi, cudaStream_t st) {
-  if (sh.K <= 4 * kBK) return launch_gemm_st<BN, B_MN_MAJOR, 2>(a, b, sh, heads, epi, st);
-  return launch_gemm_st<BN, B_MN_MAJOR, 4>(a, b, sh, heads, epi, st);
+  using PL = GemmPlan<BN, B_MN_MAJOR>;
+  auto kern = gemm_kernel<BN, B_MN_MAJOR, Epi>;
+  static std::atomic<uint64_t> done{0};
+  cudaError_t attr_err = ensure_smem_attr((const void*)kern, PL::kSmemBytes, done);
+  if (attr_err != cudaSuccess) return attr_err;
+  GemmShape s2 = sh;
+  s2.heads = heads;
+  const int64_t tiles = ((sh.M + kBM - 1) / kBM) * ((sh.N + BN - 1) / BN) * heads;
+  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  kern<<<grid, kThreads, PL::kSmemBytes, st>>>(a, b, s2, epi);
+  count_launches(1);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -374,7 +490,8 @@ cudaError_t tc_compress_append(const vmla_config& cfg, int batch, const void* x,
   if ((e = make_map_4d(&mb, w, K, N, 1, 1, (int64_t)K * 2, (int64_t)N * K * 2, (int64_t)N * K * 2, kBK, bn, 1, 128)) != cudaSuccess)
     return e;
   GemmShape sh{M, N, K, 0, wait_limit_ns(), device_status_ptr()};
-  EpiCompress epi{(bf16*)c, (bf16*)k_r, cfg.d_c, cfg.d_rope, ntok, (int64_t)cfg.window_frames * cfg.grid_h * cfg.grid_w, g, rt};
+  EpiCompress epi{(bf16*)c, (bf16*)k_r, cfg.d_c, cfg.d_rope, ntok, (int64_t)cfg.window_frames * cfg.grid_h * cfg.grid_w, g,
+                  make_rope_lookup(rt, g, cfg.chunk_frames)};
   return dispatch_bn<false>(bn, ma, mb, sh, 1, epi, st);
 }
 
@@ -391,7 +508,8 @@ cudaError_t tc_absorb_q(const vmla_config& cfg, int batch, int64_t nq, const voi
   if ((e = make_map_4d(&mb, w_uk, N, K, H, 1, (int64_t)N * 2, (int64_t)K * N * 2, (int64_t)H * K * N * 2, 64, kBK, 1, 128)) != cudaSuccess)
     return e;
   GemmShape sh{M, N, K, 1, wait_limit_ns(), device_status_ptr()};
-  EpiAbsorb epi{(bf16*)q_abs, (const bf16*)q_rope, H, cfg.d_c, cfg.d_rope, nq, g, rt};
+  EpiAbsorb epi{(bf16*)q_abs, (const bf16*)q_rope, H, cfg.d_c, cfg.d_rope, nq, g,
+                make_rope_lookup(rt, g, (int)(nq / ((int64_t)cfg.grid_h * cfg.grid_w)))};
   return dispatch_bn<true>(N, ma, mb, sh, H, epi, st);
 }
 
@@ -407,7 +525,7 @@ cudaError_t tc_value_up(const vmla_config& cfg, int batch, int64_t n_tokens, con
   if ((e = make_map_4d(&mb, w_uv, K, N, H, 1, (int64_t)K * 2, (int64_t)N * K * 2, (int64_t)H * N * K * 2, kBK, N, 1, 128)) != cudaSuccess)
     return e;
   GemmShape sh{M, N, K, 1, wait_limit_ns(), device_status_ptr()};
-  EpiValueUp epi{(bf16*)out, H, N};
+  EpiValueUp epi{RopeLookup{}, (bf16*)out, H, N};
   return dispatch_bn<false>(N, ma, mb, sh, H, epi, st);
 }
 
@@ -427,7 +545,7 @@ cudaError_t tc_dense_append(const vmla_config& cfg, int batch, const void* x, co
     return e;
   GemmShape sh{M, N, K, 0, wait_limit_ns(), device_status_ptr()};
   EpiDense epi{(bf16*)k, (bf16*)v, cfg.n_heads, cfg.d_nope, d_h, cfg.d_v, ntok,
-               (int64_t)cfg.window_frames * cfg.grid_h * cfg.grid_w, g, rt};
+               (int64_t)cfg.window_frames * cfg.grid_h * cfg.grid_w, g, make_rope_lookup(rt, g, cfg.chunk_frames)};
   return dispatch_bn<false>(bn, ma, mb, sh, 1, epi, st);
 }
 

@@ -73,8 +73,9 @@ __device__ __forceinline__ void rope_rotate_f32(const RopeTable& rt, int p, int6
   const int ax = rt.axis[p];
   const double pos = (double)(ax == 0 ? f : (ax == 1 ? i : j));
   const double two_pi = 6.283185307179586476925286766559;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
   double ang = pos * rt.inv_freq[p];
-  ang = fma(-two_pi, rint(ang / two_pi), ang);
+  ang = fma(-two_pi, rint(ang * inv_two_pi), ang);
   float sf, cf;
   sincosf((float)ang, &sf, &cf);
   *ra = a * cf - b * sf;
