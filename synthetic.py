@@ -80,3 +80,32 @@ def draw_queries(cfg: VmlaConfig, batch: int, seed: int, n_query_chunks: int = 1
     q_nope = _randn(g, (batch, nq, cfg.n_heads, cfg.d_nope), q_gain, dt)
     q_rope = _randn(g, (batch, nq, cfg.n_heads, cfg.d_rope), q_gain, dt)
     return q_nope, q_rope
+
+
+def draw_weights(cfg: VmlaConfig, seed: int):
+    """One layer's weights only, in the same order and distributions as draw_layer:
+    (W^KV_down || W^KR [d_c + d_rope, D], W^K_up [n_h, d_nope, d_c], W^V_up [n_h, d_v, d_c])."""
+    g = torch.Generator().manual_seed(int(seed))
+    dt = storage_dtype(cfg)
+    D, H = cfg.dim, cfg.n_heads
+    w_dkv_kr = _randn(g, (cfg.d_c + cfg.d_rope, D), D ** -0.5, dt)
+    w_uk = _randn(g, (H, cfg.d_nope, cfg.d_c), cfg.d_c ** -0.5, dt)
+    w_uv = _randn(g, (H, cfg.d_v, cfg.d_c), cfg.d_c ** -0.5, dt)
+    return w_dkv_kr, w_uk, w_uv
+
+
+def rollout_seed(base: int, layer: int, chunk: int) -> int:
+    """Seed of the inputs of (layer, chunk) in a streaming rollout; the layer's weights use chunk -1."""
+    return int(base) + 1_000_003 * (layer + 1) + 7919 * (chunk + 1)
+
+
+def draw_chunk(cfg: VmlaConfig, batch: int, seed: int, q_gain: float = 1.0):
+    """One streaming chunk's inputs: x [B, F*T_f, D], q^nope [B, F*T_f, n_h, d_nope],
+    q^rope [B, F*T_f, n_h, d_rope] (N(0, 1); q scaled by q_gain)."""
+    g = torch.Generator().manual_seed(int(seed))
+    dt = storage_dtype(cfg)
+    n = cfg.chunk_tokens
+    x = _randn(g, (batch, n, cfg.dim), 1.0, dt)
+    q_nope = _randn(g, (batch, n, cfg.n_heads, cfg.d_nope), q_gain, dt)
+    q_rope = _randn(g, (batch, n, cfg.n_heads, cfg.d_rope), q_gain, dt)
+    return x, q_nope, q_rope
