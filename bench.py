@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense MHA comparison arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--workload", default="layer", choices=["layer", "batch8", "dc_sweep", "rollout"],
+                    help="layer: the headline line; the others print a measurement line of their own")
     return ap.parse_args()
 
 
@@ -305,10 +307,117 @@ def run_reference(args):
 # ------------------------------------------------------------------------------------------------
 # GPU arm
 # ------------------------------------------------------------------------------------------------
+def _time(fn, reps, stream):
+    """Mean device time (ms) of fn() over reps calls, CUDA events around each, L2 not flushed."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in evs:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def run_workload(args):
+    """Measurement lines for the larger workloads (not the headline): batch-8 latent vs dense,
+    the d_c sweep at batch 16, and the 30-layer x 80-chunk streaming rollout at batch 4."""
+    from rank_latent_kv_vmla_b200 import vmla as V
+    import synthetic
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    out = {"workload": args.workload, "device": torch.cuda.get_device_name(0)}
+    clocks = ClockSampler(0)
+    if args.workload in ("batch8", "dc_sweep"):
+        B = 8 if args.workload == "batch8" else 16
+        dcs = [192] if args.workload == "batch8" else [64, 128, 192]
+        rows = []
+        clocks.start()
+        for d_c in dcs:
+            cfg = WAN.replace(d_c=d_c)
+            inp = synthetic.draw_layer(cfg, batch=B, seed=1234 + 2, n_chunks=7)
+            cache = V.LatentCache(cfg, B, device=dev)
+            w = inp.w_dkv_kr.to(dev)
+            for x in inp.x_chunks:
+                f0 = cache.frames_written
+                V.compress_append(cfg, x.to(dev), w, cache)
+            qn, qr, wuk = inp.q_nope.to(dev), inp.q_rope.to(dev), inp.w_uk.to(dev)
+            q_abs = V.absorb_q(cfg, qn, qr, wuk, f0)
+            o_lat = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_c), dtype=torch.bfloat16, device=dev)
+            for _ in range(3):
+                V.latent_attention(cfg, q_abs, cache, f0, out=o_lat)
+            ms = _time(lambda: V.latent_attention(cfg, q_abs, cache, f0, out=o_lat), 20, stream)
+            row = {"d_c": d_c, "batch": B, "latent_attention_ms": ms,
+                   "latent_tflops": attention_flops(cfg, B) / (ms * 1e-3) / 1e12,
+                   "query_tokens_per_s": B * cfg.chunk_tokens / (ms * 1e-3),
+                   "cache_bytes_per_layer": V.latent_cache_bytes(cfg, B),
+                   "cache_fraction_of_dense": V.latent_cache_bytes(cfg, B) / V.dense_cache_bytes(cfg, B)}
+            if args.workload == "batch8":
+                w_kv = synthetic.draw_dense_weights(cfg, 77).to(dev)
+                dcache = V.DenseCache(cfg, B, device=dev)
+                for x in inp.x_chunks:
+                    V.dense_append(cfg, x.to(dev), w_kv, dcache)
+                q = V.rope_q(cfg, qn, qr, f0)
+                o_d = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
+                for _ in range(3):
+                    V.dense_mha(cfg, q, dcache, f0, out=o_d)
+                dms = _time(lambda: V.dense_mha(cfg, q, dcache, f0, out=o_d), 20, stream)
+                row.update({"dense_mha_ms": dms, "dense_tflops": dense_attention_flops(cfg, B) / (dms * 1e-3) / 1e12,
+                            "attention_time_ratio_latent_over_dense": ms / dms,
+                            "dense_cache_bytes_per_layer": V.dense_cache_bytes(cfg, B)})
+                del dcache
+            rows.append(row)
+            del cache
+            torch.cuda.empty_cache()
+        out["rows"] = rows
+    else:
+        cfg, B, L, n_chunks = WAN, 4, 30, 80
+        n_sets = 3
+        sets = [tuple(t.to(dev) for t in synthetic.draw_chunk(cfg, B, synthetic.rollout_seed(9, 0, k))) for k in range(n_sets)]
+        weights = [tuple(t.to(dev) for t in synthetic.draw_weights(cfg, synthetic.rollout_seed(9, l, -1))) for l in range(L)]
+        dense_w = [synthetic.draw_dense_weights(cfg, 500 + l).to(dev) for l in range(L)]
+        res = {}
+        clocks.start()
+        for path in ("latent", "dense"):
+            caches = [V.LatentCache(cfg, B, device=dev) if path == "latent" else V.DenseCache(cfg, B, device=dev)
+                      for _ in range(L)]
+            bufs = {"q_abs": torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_qk), dtype=torch.bfloat16, device=dev),
+                    "o_latent": torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_c), dtype=torch.bfloat16, device=dev),
+                    "o": torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)}
+            dq = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_h), dtype=torch.bfloat16, device=dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record(stream)
+            for k in range(n_chunks):
+                x, qn, qr = sets[k % n_sets]
+                for l in range(L):
+                    if path == "latent":
+                        wd, wuk, wuv = weights[l]
+                        V.layer_step(cfg, x, qn, qr, wd, wuk, wuv, caches[l], bufs)
+                    else:
+                        f0 = caches[l].frames_written
+                        V.dense_append(cfg, x, dense_w[l], caches[l], f0)
+                        V.rope_q(cfg, qn, qr, f0, out=dq)
+                        V.dense_mha(cfg, dq, caches[l], f0, out=bufs["o"])
+            b.record(stream)
+            torch.cuda.synchronize()
+            res[path] = {"total_s": a.elapsed_time(b) / 1e3,
+                         "cache_bytes_all_layers": sum(c.nbytes() for c in caches)}
+            del caches
+            torch.cuda.empty_cache()
+        res["speedup_latent_over_dense"] = res["dense"]["total_s"] / res["latent"]["total_s"]
+        res["latent"]["attention_tflops"] = attention_flops(cfg, B) * L * n_chunks / res["latent"]["total_s"] / 1e12
+        out.update({"layers": L, "chunks": n_chunks, "batch": B, "frames": n_chunks * cfg.chunk_frames, **res})
+    out["clocks"] = clocks.stop()
+    assert V.device_status() == 0
+    print(json.dumps(out), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload != "layer":
+        return run_workload(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     rank, world, local = dist_setup("nccl")
