@@ -112,8 +112,8 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   uint64_t* kv_full = bars + 1;           // NST
   uint64_t* kv_empty = kv_full + NST;     // NST
   uint64_t* s_full = kv_empty + NST;      // NS
-  uint64_t* p_ready = s_full + NS;        // NS
-  uint64_t* pv_done = p_ready + NS;       // NS: P V of a tile of that S buffer completed
+  uint64_t* p_ready = s_full + NS;        // [NS][2]: P of the first / second half of the tile's keys
+  uint64_t* pv_done = p_ready + 2 * NS;   // NS: P V of a tile of that S buffer completed
   uint64_t* drain = pv_done + NS;         // 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -135,7 +135,12 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   if (threadIdx.x == 0) {
     mbar_init(bar_q, Q_TMEM ? 128 : 1);
     for (int s = 0; s < NST; ++s) { mbar_init(kv_full + s, 1); mbar_init(kv_empty + s, 1); }
-    for (int s = 0; s < NS; ++s) { mbar_init(s_full + s, 1); mbar_init(p_ready + s, 128); mbar_init(pv_done + s, 1); }
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(s_full + s, 1);
+      mbar_init(p_ready + 2 * s, 128);
+      mbar_init(p_ready + 2 * s + 1, 128);
+      mbar_init(pv_done + s, 1);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -191,13 +196,18 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       const uint32_t q_base = smem_u32(sQ);
       const uint32_t kv_base = smem_u32(sKV);
       bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, 2, p.limit_ns);
+      // P V of tile jp in two halves of the keys: the first half's MMAs run while the softmax warps
+      // still produce the second half's P
       auto issue_pv = [&](int jp) -> bool {
         const int bp = jp % NS;
-        if (!mbar_wait(p_ready + bp, (jp / NS) & 1, abort_flag, p.status, 3, p.limit_ns)) return false;
-        tc_fence_after();
         const uint32_t v_base = kv_base + (jp % NST) * PL::kStageBytes + PL::kVOff;
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k) {
+          if (k == 0 || k == BN / 32) {
+            if (!mbar_wait(p_ready + 2 * bp + (k ? 1 : 0), (jp / NS) & 1, abort_flag, p.status, 3, p.limit_ns))
+              return false;
+            tc_fence_after();
+          }
           // V tile [BN keys][NPV] as MN-major operand: 8-key groups 1024 B apart (SBO), 64-column
           // boxes BN*128 B apart (LBO, the ones box being the last); a K step of 16 keys is 2048 B.
           const uint64_t vdesc = smem_desc(v_base + k * 2048, PL::kBox, 1024, kSwizzle128B);
@@ -375,6 +385,11 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st8(tmem + lane_base + bj * BN + c * 8, pk);
+        if (c == BN / 32 - 1) {                       // first half of the keys: release it to P V
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(p_ready + 2 * bj);
+        }
       }
       if (!ONES) {
         fadd2(ls[0], ls[1], ls[4], ls[5]);
@@ -384,7 +399,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_ready + bj);
+      mbar_arrive(p_ready + 2 * bj + 1);
     }
     bool fin = ok && mbar_wait(drain, 0, abort_flag, p.status, 7, p.limit_ns);
     fin = __all_sync(0xffffffffu, fin && !*abort_flag);
