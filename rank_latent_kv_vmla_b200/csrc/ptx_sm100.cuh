@@ -312,5 +312,32 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^x for a pair of arguments on the FMA and integer pipes, leaving MUFU free.  Write x = n + f with n
+// the nearest integer and |f| <= 1/2: adding 1.5 * 2^23 rounds x to n and leaves n in the low mantissa
+// bits of the sum.  2^f comes from a cubic fitted (Lawson's iteration) for least maximum relative
+// error on [-1/2, 1/2]: 7.5e-5, well under bf16's half-ulp of 2^-9.  Multiplying the sum's bits by 2^23
+// moves n (mod 2^9) into the exponent field, and one integer add scales 2^f by 2^n.  Arguments are
+// clamped to >= -125 first, so the exponent stays normal (2^-125 ~ 2.4e-38 stands in for smaller
+// results and for -inf); callers pass x <= 120.
+__device__ __forceinline__ void exp2_poly2(float& p0, float& p1, float x0, float x1) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99992805719375610f, c1 = 0.69326096773147583f, c2 = 0.24261112511157990f,
+                  c3 = 0.05517166852951050f;
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  float t0 = kShift, t1 = kShift;
+  fadd2(t0, t1, x0, x1);                              // t = 1.5 * 2^23 + n
+  float r0 = -kShift, r1 = -kShift;
+  fadd2(r0, r1, t0, t1);                              // n
+  float f0, f1;
+  ffma2(f0, f1, r0, r1, -1.f, -1.f, x0, x1);          // f = x - n, exact
+  float q0, q1;
+  ffma2(q0, q1, f0, f1, c3, c3, c2, c2);
+  ffma2(q0, q1, q0, q1, f0, f1, c1, c1);
+  ffma2(q0, q1, q0, q1, f0, f1, c0, c0);              // 2^f
+  p0 = __uint_as_float(__float_as_uint(t0) * (1u << 23) + __float_as_uint(q0));
+  p1 = __uint_as_float(__float_as_uint(t1) * (1u << 23) + __float_as_uint(q1));
+}
+
 }  // namespace sm100
 }  // namespace vmla

@@ -38,6 +38,12 @@ constexpr int kThreads = 192;          // 6 warps
 constexpr int kBlockM = 128;           // query rows per CTA
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Of the 8 score pairs in each 16-key chunk, this many take 2^x from the FMA-pipe polynomial
+// (exp2_poly2) and the rest from MUFU.EX2, which one warp per SM sub-partition would otherwise saturate.
+#ifndef VMLA_EXP2_POLY_PAIRS
+#define VMLA_EXP2_POLY_PAIRS 2
+#endif
+constexpr int kPolyPairs = VMLA_EXP2_POLY_PAIRS;
 
 struct AttnParams {
   const void* q;         // query rows (used when Q is kept in TMEM)
@@ -380,7 +386,13 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         for (int i = 0; i < 8; ++i) {
           float x0, x1;
           ffma2(x0, x1, sr[c * 16 + 2 * i], sr[c * 16 + 2 * i + 1], sc, sc, neg_m, neg_m);
-          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          float p0, p1;
+          if (i < kPolyPairs) {
+            exp2_poly2(p0, p1, x0, x1);
+          } else {
+            p0 = fast_exp2(x0);
+            p1 = fast_exp2(x1);
+          }
           if (!ONES) fadd2(ls[(2 * i) & 7], ls[(2 * i + 1) & 7], p0, p1);
           pk[i] = pack_bf16x2(p0, p1);
         }
