@@ -11,6 +11,7 @@ Sources (page title, section):
   [TS-P]  same title, gist.science technical summary, "Problem definition" section.
   [TS-M1] .. [TS-M4]  same summary, "Method: VideoMLA" items 1-4 (shared latent, on-demand
           reconstruction, decoupled 3D-RoPE, memory reduction).
+  [TS-R]  same summary, "Results" section, "Scalability" item (batch size at a fixed memory budget).
 
 Readings where the pages are silent (each one is listed with its reason in the design notes):
   * the head-shared key k^R_t is projected from x_t by its own matrix W^KR (not from c_t);
@@ -21,7 +22,11 @@ Readings where the pages are silent (each one is listed with its reason in the d
   * the window counts frames and includes the current chunk: query chunk k of a call sees key frames
     [max(0, hi_k - W), hi_k) with hi_k the end frame of its chunk (bidirectional inside a chunk,
     causal across chunks);
-  * softmax scale 1/sqrt(d_nope + d_rope); d_v = d_h.
+  * softmax scale 1/sqrt(d_nope + d_rope); d_v = d_h;
+  * few-step generation: a chunk is denoised over several steps and its own keys and values are
+    recomputed from each step's features, replacing the chunk's entries in place (older frames kept);
+  * batch capacity: the bytes that grow with the batch are every layer's cache plus one layer step's
+    tensors (reused across layers) plus caller-given activations; weights are fixed.
 
 Parity status: every function here is pinned by tests/test_oracle_pins.py (closed-form cache
 arithmetic printed on the pages, RoPE invariants and the textbook complex-number 1-D RoPE, brute-force
@@ -245,6 +250,16 @@ class History:
         self.k_r = np.concatenate([self.k_r, k_r])
         self.frames = np.concatenate([self.frames, frames])
 
+    def rewrite_newest(self, c: np.ndarray, k_r: np.ndarray, frames: np.ndarray):
+        """One denoising step of a few-step chunk: the newest tokens (whose frames must be ``frames``)
+        get the entries computed from this step's features; every older entry is kept.  [TS-P] names
+        Self-Forcing-style training; recomputing the chunk in place is the reading."""
+        n = len(frames)
+        if n == 0 or n > len(self.frames) or not np.array_equal(self.frames[-n:], frames):
+            raise ValueError("rewrite must cover exactly the newest tokens")
+        self.c = np.concatenate([self.c[:-n], c])
+        self.k_r = np.concatenate([self.k_r[:-n], k_r])
+
 
 def build_history(x_chunks, w_dkv_kr, b: int, *, d_c, d_rope, chunk_frames, grid_h, grid_w, pairs,
                   theta) -> History:
@@ -281,3 +296,59 @@ def layer_reference(hist: History, q_nope, q_rope, w_uk, w_uv, *, first_frame, q
     o_latent = p @ hist.c
     q_abs = absorbed_query(np.asarray(q_nope, F64)[rows], q_r, w_uk)
     return {"o": o, "o_latent": o_latent, "lse": lse, "q_abs": q_abs, "mask": mask}
+
+
+# ---------------------------------------------------------------------------------------------------
+# Batch capacity at a fixed memory budget  [TS-R], [TS-M4]
+# ---------------------------------------------------------------------------------------------------
+def step_tensors(batch: int, *, dim, n_heads, d_nope, d_rope, d_c, d_v, tokens_per_chunk, dense):
+    """Shapes of the tensors one layer step holds for ``batch`` sequences (reused by every layer):
+    the chunk features and, latent path, q^nope, q^rope, the absorbed query, the latent output and the
+    output; dense path, the query and the output."""
+    B, N, H = batch, tokens_per_chunk, n_heads
+    if dense:
+        return {"x": (B, N, dim), "q": (B, N, H, d_nope + d_rope), "out": (B, N, H, d_v)}
+    return {"x": (B, N, dim), "q_nope": (B, N, H, d_nope), "q_rope": (B, N, H, d_rope),
+            "q_abs": (B, N, H, d_c + d_rope), "out_latent": (B, N, H, d_c), "out": (B, N, H, d_v)}
+
+
+def layer_weights(*, dim, n_heads, d_nope, d_rope, d_c, d_v, dense):
+    """Shapes of one layer's attention-path weights: W^KV_down with W^KR stacked, W^K_up and W^V_up
+    per head [TS-M1, TS-M2, TS-M3]; dense: per-head K and V projections."""
+    if dense:
+        return {"w_kv": (n_heads * (d_nope + d_rope + d_v), dim)}
+    return {"w_dkv_kr": (d_c + d_rope, dim), "w_uk": (n_heads, d_nope, d_c), "w_uv": (n_heads, d_v, d_c)}
+
+
+def memory_bytes(batch: int, *, n_layers, window_tokens, elt_bytes, fixed_bytes, extra_bytes_per_seq,
+                 dense, **shape) -> int:
+    """Every byte held at once for ``batch`` sequences: each layer's cache (per token the dense
+    2*n_h*d_h or the latent d_c + d_rope scalars [TS-M4]), each layer's weights, one layer step's tensors,
+    the caller's fixed bytes and its per-sequence extra bytes."""
+    if dense:
+        per_token = shape["n_heads"] * (shape["d_nope"] + shape["d_rope"] + shape["d_v"])
+    else:
+        per_token = latent_scalars_per_token(shape["d_c"], shape["d_rope"])
+    scalars = n_layers * batch * window_tokens * per_token
+    scalars += n_layers * sum(int(np.prod(v)) for v in layer_weights(dense=dense, **{
+        k: shape[k] for k in ("dim", "n_heads", "d_nope", "d_rope", "d_c", "d_v")}).values())
+    scalars += sum(int(np.prod(v)) for v in step_tensors(batch, dense=dense, **shape).values())
+    return scalars * elt_bytes + fixed_bytes + batch * extra_bytes_per_seq
+
+
+def batch_capacity(budget_bytes: int, **kw) -> int:
+    """Largest batch whose memory_bytes fits ``budget_bytes`` (0 if none): memory grows with the batch,
+    so double until it no longer fits, then bisect [TS-R]."""
+    if memory_bytes(0, **kw) > budget_bytes:
+        return 0
+    hi = 1
+    while memory_bytes(hi, **kw) <= budget_bytes:
+        hi *= 2
+    lo = hi // 2                                     # fits; hi does not
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if memory_bytes(mid, **kw) <= budget_bytes:
+            lo = mid
+        else:
+            hi = mid
+    return lo

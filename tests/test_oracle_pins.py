@@ -382,3 +382,94 @@ def test_layer_reference_row_sampling_is_consistent():
     part = _ref(cfg, inp, hist, 2, rows=rows)
     for key in ("o", "o_latent", "lse", "q_abs"):
         np.testing.assert_array_equal(part[key], full[key][rows])
+
+
+# ------------------------------------------------------------------------------------------------
+# Few-step generation: in-place rewrite of the newest chunk
+# ------------------------------------------------------------------------------------------------
+def test_rewrite_newest_equals_history_built_with_that_chunk():
+    """Rewriting the newest chunk with x' gives exactly the history built from the chunk list whose last
+    entry is x'; rewriting with the same x changes nothing; only the newest tokens can be rewritten."""
+    cfg = TINY
+    inp = synthetic.draw_layer(cfg, batch=1, seed=91, n_chunks=5)
+    xs = [_f64(x) for x in inp.x_chunks]
+    w = _f64(inp.w_dkv_kr)
+    kw = _tiny_kwargs(cfg)
+    hist = O.build_history(xs[:4], w, 0, **kw)
+    before_c, before_k = hist.c.copy(), hist.k_r.copy()
+    pos = O.token_positions(3 * cfg.chunk_frames, cfg.chunk_tokens, cfg.grid_h, cfg.grid_w)
+    c, k_r = O.compress(xs[3][0], w, cfg.d_c, pos, kw["pairs"], cfg.rope_theta)
+    hist.rewrite_newest(c, k_r, pos[:, 0])
+    np.testing.assert_array_equal(hist.c, before_c)
+    np.testing.assert_array_equal(hist.k_r, before_k)
+    c2, k2 = O.compress(xs[4][0], w, cfg.d_c, pos, kw["pairs"], cfg.rope_theta)
+    hist.rewrite_newest(c2, k2, pos[:, 0])
+    other = O.build_history(xs[:3] + [xs[4]], w, 0, **kw)
+    np.testing.assert_array_equal(hist.c, other.c)
+    np.testing.assert_array_equal(hist.k_r, other.k_r)
+    np.testing.assert_array_equal(hist.frames, other.frames)
+    n = cfg.chunk_tokens
+    np.testing.assert_array_equal(hist.c[:-n], before_c[:-n])
+    old_pos = O.token_positions(2 * cfg.chunk_frames, n, cfg.grid_h, cfg.grid_w)
+    with pytest.raises(ValueError):
+        hist.rewrite_newest(c2, k2, old_pos[:, 0])
+
+
+# ------------------------------------------------------------------------------------------------
+# Batch capacity at a fixed memory budget
+# ------------------------------------------------------------------------------------------------
+def _wan_capacity_kwargs(**over):
+    kw = dict(n_layers=30, window_tokens=WAN.window_tokens, elt_bytes=2, fixed_bytes=0,
+              extra_bytes_per_seq=0, dim=WAN.dim, n_heads=WAN.n_heads, d_nope=WAN.d_nope,
+              d_rope=WAN.d_rope, d_c=WAN.d_c, d_v=WAN.d_v, tokens_per_chunk=WAN.chunk_tokens)
+    kw.update(over)
+    return kw
+
+
+def test_capacity_cache_terms_match_printed_figures():
+    """The per-sequence growth of memory_bytes, less one layer step's tensors, is the cache: the dense
+    one is the printed ~6.0 GB (30 layers, bf16, 21 frames), the latent one 7.3 % of it (92.7 %)."""
+    g = json.load(open(GOLDEN))
+    per_seq = {}
+    for dense in (False, True):
+        kw = _wan_capacity_kwargs(dense=dense)
+        grow = O.memory_bytes(2, **kw) - O.memory_bytes(1, **kw)
+        step = (O.memory_bytes(1, **kw) - O.memory_bytes(0, **kw)) - grow    # 0: linear in the batch
+        assert step == 0
+        shape = {k: kw[k] for k in ("dim", "n_heads", "d_nope", "d_rope", "d_c", "d_v", "tokens_per_chunk")}
+        tensors = sum(int(np.prod(v)) for v in O.step_tensors(1, dense=dense, **shape).values()) * 2
+        per_seq[dense] = grow - tensors
+    assert round(per_seq[True] / 1e9, 1) == g["dense_cache_gb_21_frames"]["value"]
+    red = 100 * (1 - per_seq[False] / per_seq[True])
+    assert round(red, 1) == g["reduction_percent"]["value"]
+    # the printed batch ratios lie below the cache-only ratio 3072 / 224
+    assert g["batch_ratio_dc192"]["value"] < per_seq[True] / per_seq[False]
+    assert g["batch_ratio_lower_dc_max"]["value"] < 3072 / (64 + 32)
+
+
+def test_capacity_search_is_exact_and_matches_a_linear_scan():
+    kw = _wan_capacity_kwargs(fixed_bytes=3_000_000_000, extra_bytes_per_seq=123_456_789)
+    for dense in (False, True):
+        for k in (0, 1, 7, 29, 300):
+            exact = O.memory_bytes(k, dense=dense, **kw)
+            assert O.batch_capacity(exact, dense=dense, **kw) == k
+            if k > 0:
+                assert O.batch_capacity(exact - 1, dense=dense, **kw) == k - 1
+    assert O.batch_capacity(O.memory_bytes(0, dense=False, **kw) - 1, dense=False, **kw) == 0
+    tiny = dict(n_layers=2, window_tokens=TINY.window_tokens, elt_bytes=4, fixed_bytes=1000,
+                extra_bytes_per_seq=10, dim=TINY.dim, n_heads=TINY.n_heads, d_nope=TINY.d_nope,
+                d_rope=TINY.d_rope, d_c=TINY.d_c, d_v=TINY.d_v, tokens_per_chunk=TINY.chunk_tokens)
+    for dense in (False, True):
+        for budget in range(0, 400_000, 9_973):
+            scan = 0
+            while O.memory_bytes(scan + 1, dense=dense, **tiny) <= budget:
+                scan += 1
+            if O.memory_bytes(0, dense=dense, **tiny) > budget:
+                scan = 0
+            assert O.batch_capacity(budget, dense=dense, **tiny) == scan
+
+
+def test_capacity_grows_as_the_latent_shrinks():
+    caps = [O.batch_capacity(180 * 10**9, dense=False, **_wan_capacity_kwargs(d_c=d)) for d in (64, 128, 192)]
+    dense = O.batch_capacity(180 * 10**9, dense=True, **_wan_capacity_kwargs())
+    assert caps[0] > caps[1] > caps[2] > dense > 0
