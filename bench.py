@@ -48,7 +48,8 @@ def parse():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense MHA comparison arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
-    ap.add_argument("--workload", default="layer", choices=["layer", "batch8", "dc_sweep", "rollout"],
+    ap.add_argument("--workload", default="layer", choices=["layer", "batch8", "dc_sweep", "rollout", "fewstep",
+                                                            "capacity"],
                     help="layer: the headline line; the others print a measurement line of their own")
     return ap.parse_args()
 
@@ -318,9 +319,109 @@ def _time(fn, reps, stream):
     return statistics.mean(a.elapsed_time(b) for a, b in evs)
 
 
+def _fewstep_workload(V, synthetic, dev, stream, clocks, batch=1, n_chunks=14, n_denoise=4):
+    """One Wan layer streaming n_chunks chunks, each denoised over n_denoise steps: the first step
+    appends the chunk, the others rewrite it in place; every step attends with its own queries
+    (latent: compress -> absorb -> attention -> value-up; dense: project -> rope -> MHA)."""
+    cfg, B = WAN, batch
+    sets = [tuple(t.to(dev) for t in synthetic.draw_chunk(cfg, B, synthetic.rollout_seed(11, 0, k)))
+            for k in range(n_denoise)]
+    wd, wuk, wuv = (t.to(dev) for t in synthetic.draw_weights(cfg, 12))
+    w_kv = synthetic.draw_dense_weights(cfg, 13).to(dev)
+    q_abs = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_qk), dtype=torch.bfloat16, device=dev)
+    o_lat = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_c), dtype=torch.bfloat16, device=dev)
+    o = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
+    dq = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_h), dtype=torch.bfloat16, device=dev)
+    res = {}
+    clocks.start()
+    for path in ("latent", "dense"):
+        cache = V.LatentCache(cfg, B, device=dev) if path == "latent" else V.DenseCache(cfg, B, device=dev)
+        evs = []
+        for k in range(n_chunks):
+            for s in range(n_denoise):
+                x, qn, qr = sets[s]
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                if path == "latent":
+                    if s == 0:
+                        f0 = cache.frames_written
+                        V.compress_append(cfg, x, wd, cache)
+                    else:
+                        V.compress_rewrite(cfg, x, wd, cache)
+                    V.absorb_q(cfg, qn, qr, wuk, f0, out=q_abs)
+                    V.latent_attention(cfg, q_abs, cache, f0, out=o_lat)
+                    V.value_up(cfg, o_lat, wuv, out=o)
+                else:
+                    if s == 0:
+                        f0 = cache.frames_written
+                        V.dense_append(cfg, x, w_kv, cache)
+                    else:
+                        V.dense_rewrite(cfg, x, w_kv, cache)
+                    V.rope_q(cfg, qn, qr, f0, out=dq)
+                    V.dense_mha(cfg, dq, cache, f0, out=o)
+                b.record(stream)
+                evs.append((k, a, b))
+        torch.cuda.synchronize()
+        # steady state: chunks whose window is full (frame f0 + F >= W)
+        full = [a.elapsed_time(b) for k, a, b in evs if (k + 1) * cfg.chunk_frames >= cfg.window_frames]
+        ms = statistics.mean(full)
+        fl = attention_flops(cfg, B) if path == "latent" else dense_attention_flops(cfg, B)
+        res[path] = {"ms_per_denoising_step": ms, "attention_tflops_per_step_time": fl / (ms * 1e-3) / 1e12,
+                     "steps_timed": len(full), "total_ms_all_steps": sum(a.elapsed_time(b) for _, a, b in evs)}
+        del cache
+        torch.cuda.empty_cache()
+    res["step_time_ratio_latent_over_dense"] = res["latent"]["ms_per_denoising_step"] / res["dense"]["ms_per_denoising_step"]
+    return {"batch": B, "chunks": n_chunks, "denoising_steps_per_chunk": n_denoise, **res}
+
+
+def _capacity_workload(V, synthetic, dev, clocks, budget=60 * 10**9, n_layers=30):
+    """Largest batch for 30 Wan layers under a 60 GB budget, latent (d_c 64 / 128 / 192) and dense,
+    from the planner; for d_c = 192 and dense the planned caches of all layers are then allocated and
+    one layer step runs at that batch, with the device's peak allocation recorded."""
+    rows = []
+    clocks.start()
+    for name, cfg, dense in (("latent_dc64", WAN.replace(d_c=64), False),
+                             ("latent_dc128", WAN.replace(d_c=128), False),
+                             ("latent_dc192", WAN, False), ("dense", WAN, True)):
+        plan = V.plan_capacity(cfg, n_layers, budget, dense=dense)
+        row = {"path": name, **plan}
+        if name in ("latent_dc192", "dense"):
+            B = plan["max_batch"]
+            torch.cuda.empty_cache()
+            torch.cuda.reset_peak_memory_stats()
+            x, qn, qr = (t.to(dev) for t in synthetic.draw_chunk(cfg, B, 21))
+            if dense:
+                w_kv = synthetic.draw_dense_weights(cfg, 22).to(dev)
+                caches = [V.DenseCache(cfg, B, device=dev) for _ in range(n_layers)]
+                ws = [w_kv] * n_layers
+            else:
+                wd, wuk, wuv = (t.to(dev) for t in synthetic.draw_weights(cfg, 22))
+                caches = [V.LatentCache(cfg, B, device=dev) for _ in range(n_layers)]
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record()
+            if dense:
+                V.dense_append(cfg, x, w_kv, caches[0])
+                out = V.dense_mha(cfg, V.rope_q(cfg, qn, qr, 0), caches[0], 0)
+            else:
+                out = V.layer_step(cfg, x, qn, qr, wd, wuk, wuv, caches[0])
+            t1.record()
+            torch.cuda.synchronize()
+            row.update({"allocated_batch": B, "peak_allocated_bytes": torch.cuda.max_memory_allocated(),
+                        "one_layer_step_ms": t0.elapsed_time(t1), "output_finite": bool(torch.isfinite(out).all())})
+            del caches, out, x, qn, qr
+            torch.cuda.empty_cache()
+        rows.append(row)
+    by = {r["path"]: r["max_batch"] for r in rows}
+    return {"budget_bytes": budget, "n_layers": n_layers, "rows": rows,
+            "batch_ratio_dc192_over_dense": by["latent_dc192"] / max(by["dense"], 1),
+            "batch_ratio_dc64_over_dense": by["latent_dc64"] / max(by["dense"], 1)}
+
+
 def run_workload(args):
     """Measurement lines for the larger workloads (not the headline): batch-8 latent vs dense,
-    the d_c sweep at batch 16, and the 30-layer x 80-chunk streaming rollout at batch 4."""
+    the d_c sweep at batch 16, the 30-layer x 80-chunk streaming rollout at batch 4, few-step
+    generation (4 denoising steps per chunk) and the batch capacity at a 60 GB budget."""
     from rank_latent_kv_vmla_b200 import vmla as V
     import synthetic
     dev = torch.device("cuda", 0)
@@ -369,6 +470,10 @@ def run_workload(args):
             del cache
             torch.cuda.empty_cache()
         out["rows"] = rows
+    elif args.workload == "fewstep":
+        out.update(_fewstep_workload(V, synthetic, dev, stream, clocks))
+    elif args.workload == "capacity":
+        out.update(_capacity_workload(V, synthetic, dev, clocks))
     else:
         cfg, B, L, n_chunks = WAN, 4, 30, 80
         n_sets = 3

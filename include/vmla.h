@@ -104,6 +104,16 @@ typedef struct {
 VMLA_API vmla_status vmla_compress_append(const vmla_config* cfg, const void* x, const void* w_dkv_kr,
                                  int64_t first_frame, vmla_cache* cache, void* stream);
 
+/* Few-step generation: recompute the newest chunk's cache rows in place.  Streaming video diffusion
+ * denoises each chunk over several steps (the technical summary's Problem definition names
+ * Self-Forcing-style training); at every step the chunk's own keys come from that step's features,
+ * and the last rewrite, with the clean features, is what stays in the window.  This call does what
+ * vmla_compress_append does for the frames frames_written-F .. frames_written-1 (same x, w_dkv_kr
+ * layouts), without advancing frames_written and without evicting anything: the frames the chunk's
+ * first append evicted are outside its window.  Requires frames_written >= F. */
+VMLA_API vmla_status vmla_compress_rewrite(const vmla_config* cfg, const void* x, const void* w_dkv_kr,
+                                           vmla_cache* cache, void* stream);
+
 /* Absorbed query (VideoMLA, Method item 2 "on-demand reconstruction" with W^K_up folded into the
  * query; item 3 for the rotated part).
  *   q_nope [batch, Nq, n_heads, d_nope], q_rope [batch, Nq, n_heads, d_rope],
@@ -148,6 +158,11 @@ VMLA_API vmla_status vmla_rope_q(const vmla_config* cfg, int32_t batch, int32_t 
 VMLA_API vmla_status vmla_dense_append(const vmla_config* cfg, const void* x, const void* w_kv,
                               int64_t first_frame, vmla_dense_cache* cache, void* stream);
 
+/* Dense counterpart of vmla_compress_rewrite: recompute the newest chunk's keys and values in place
+ * (frames frames_written-F ..), frames_written unchanged.  Requires frames_written >= F. */
+VMLA_API vmla_status vmla_dense_rewrite(const vmla_config* cfg, const void* x, const void* w_kv,
+                                        vmla_dense_cache* cache, void* stream);
+
 /* Dense multi-head attention with the same window / block-causal rule as vmla_latent_attention.
  *   q [batch, Nq, n_heads, d_h] -> out [batch, Nq, n_heads, d_v], lse [batch, Nq, n_heads] (or NULL). */
 VMLA_API vmla_status vmla_dense_mha(const vmla_config* cfg, const void* q, const vmla_dense_cache* cache,
@@ -171,6 +186,27 @@ VMLA_API vmla_status vmla_device_status(void* stream, int32_t* code);
  * and dense (n_heads*(d_h + d_v) per token), in the storage type of cfg->dtype.  -1 on a bad cfg. */
 VMLA_API int64_t vmla_latent_cache_bytes(const vmla_config* cfg, int32_t batch);
 VMLA_API int64_t vmla_dense_cache_bytes(const vmla_config* cfg, int32_t batch);
+
+/* Largest batch that fits a fixed memory budget (the technical summary's Results, "Scalability": at a
+ * fixed B200 memory budget the latent cache admits a much larger batch than dense MHA).  For a model of
+ * n_layers attention layers of this shape (dense = 0: latent path, 1: dense MHA path):
+ *   per sequence  cache   n_layers * W*T_f * (d_c + d_rope)  or  n_layers * W*T_f * n_heads*(d_h + d_v)
+ *                 buffers the tensors of one layer step, reused across layers (x [F*T_f, dim] and,
+ *                         latent: q_nope, q_rope, q_abs, out_latent, out; dense: q, out)
+ *                 + extra_bytes_per_seq (activations outside this library)
+ *   fixed         this library's weights for n_layers layers (latent: w_dkv_kr, w_uk, w_uv; dense:
+ *                 w_kv) + fixed_bytes (the rest of the model)
+ * all in the storage type of cfg->dtype.  out->max_batch = floor((budget - fixed) / per sequence),
+ * 0 when the fixed bytes alone exceed the budget.  Host-only; launches nothing. */
+typedef struct {
+  int64_t max_batch;
+  int64_t cache_bytes_per_seq;   /* all layers' cache of one sequence */
+  int64_t buffer_bytes_per_seq;  /* one layer step's tensors for one sequence */
+  int64_t weight_bytes;          /* this library's weights, all layers */
+} vmla_capacity;
+VMLA_API vmla_status vmla_plan_capacity(const vmla_config* cfg, int32_t n_layers, int32_t dense,
+                                        int64_t budget_bytes, int64_t fixed_bytes,
+                                        int64_t extra_bytes_per_seq, vmla_capacity* out);
 
 /* Set the bound of every device-side wait of later launches to `ms` milliseconds (default 1000) and
  * return the previous bound; ms <= 0 only returns the current bound.  A wait that runs out makes the

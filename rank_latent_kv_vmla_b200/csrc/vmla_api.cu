@@ -171,8 +171,64 @@ int64_t vmla_dense_cache_bytes(const vmla_config* cfg, int32_t batch) {
          (cfg->d_nope + cfg->d_rope + cfg->d_v) * elt;
 }
 
-vmla_status vmla_compress_append(const vmla_config* cfg, const void* x, const void* w_dkv_kr,
-                                 int64_t first_frame, vmla_cache* cache, void* stream) {
+vmla_status vmla_plan_capacity(const vmla_config* cfg, int32_t n_layers, int32_t dense,
+                               int64_t budget_bytes, int64_t fixed_bytes, int64_t extra_bytes_per_seq,
+                               vmla_capacity* out) {
+  vmla_status s = check_config(cfg);
+  if (s != VMLA_OK) return s;
+  if (!out) return fail(VMLA_ERR_INVALID_ARG, "out is NULL");
+  if (n_layers <= 0) return fail(VMLA_ERR_INVALID_ARG, "n_layers must be >= 1");
+  if (budget_bytes < 0 || fixed_bytes < 0 || extra_bytes_per_seq < 0)
+    return fail(VMLA_ERR_INVALID_ARG, "budget, fixed and extra bytes must be >= 0");
+  const int64_t elt = cfg->dtype == VMLA_BF16 ? 2 : 4;
+  const int64_t H = cfg->n_heads, D = cfg->dim, dh = cfg->d_nope + cfg->d_rope, dv = cfg->d_v;
+  const int64_t nq = (int64_t)cfg->chunk_frames * cfg->grid_h * cfg->grid_w;
+  const int64_t nk = (int64_t)cfg->window_frames * cfg->grid_h * cfg->grid_w;
+  int64_t cache_tok, buffers, weights;
+  if (dense) {
+    cache_tok = H * (dh + dv);
+    buffers = nq * D + nq * H * dh + nq * H * dv;                               // x, q, out
+    weights = H * (dh + dv) * D;                                                // w_kv
+  } else {
+    const int64_t dc = cfg->d_c, dr = cfg->d_rope;
+    cache_tok = dc + dr;
+    buffers = nq * D + nq * H * cfg->d_nope + nq * H * dr + nq * H * (dc + dr)  // x, q_nope, q_rope, q_abs
+              + nq * H * dc + nq * H * dv;                                      // out_latent, out
+    weights = (dc + dr) * D + H * cfg->d_nope * dc + H * dv * dc;               // w_dkv_kr, w_uk, w_uv
+  }
+  out->cache_bytes_per_seq = (int64_t)n_layers * nk * cache_tok * elt;
+  out->buffer_bytes_per_seq = buffers * elt;
+  out->weight_bytes = (int64_t)n_layers * weights * elt;
+  const int64_t per_seq = out->cache_bytes_per_seq + out->buffer_bytes_per_seq + extra_bytes_per_seq;
+  const int64_t room = budget_bytes - fixed_bytes - out->weight_bytes;
+  out->max_batch = room > 0 ? room / per_seq : 0;
+  return VMLA_OK;
+}
+
+namespace {
+
+// Compress the chunk of frames first_frame .. first_frame+F-1 into its ring rows (shared by append and
+// rewrite; the caller has checked first_frame against the cache).
+vmla_status compress_chunk(const vmla_config* cfg, const void* x, const void* w_dkv_kr,
+                           int64_t first_frame, vmla_cache* cache, void* stream) {
+  const FrameGeom g = make_geom(*cfg, first_frame);
+  const RopeTable rt = make_rope_table(*cfg);
+  cudaError_t e;
+  if (cfg->dtype == VMLA_F32) {
+    e = simt_compress_append<float>(*cfg, cache->batch, (const float*)x, (const float*)w_dkv_kr, g,
+                                    rt, (float*)cache->c, (float*)cache->k_r, as_stream(stream));
+  } else {
+    vmla_status s = tc_check_compress(*cfg);
+    if (s != VMLA_OK) return fail(s, "%s", tc_last_reason());
+    e = tc_compress_append(*cfg, cache->batch, x, w_dkv_kr, g, rt, cache->c, cache->k_r,
+                           as_stream(stream));
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "compress launch");
+  return VMLA_OK;
+}
+
+vmla_status check_compress_args(const vmla_config* cfg, const void* x, const void* w_dkv_kr,
+                                const vmla_cache* cache) {
   vmla_status s = check_config(cfg);
   if (s != VMLA_OK) return s;
   if (!cache) return fail(VMLA_ERR_INVALID_ARG, "cache is NULL");
@@ -181,24 +237,32 @@ vmla_status vmla_compress_append(const vmla_config* cfg, const void* x, const vo
   VMLA_CHECK_PTR(cache->c);
   VMLA_CHECK_PTR(cache->k_r);
   if (cache->batch <= 0) return fail(VMLA_ERR_INVALID_ARG, "cache->batch must be >= 1");
+  return VMLA_OK;
+}
+
+}  // namespace
+
+vmla_status vmla_compress_append(const vmla_config* cfg, const void* x, const void* w_dkv_kr,
+                                 int64_t first_frame, vmla_cache* cache, void* stream) {
+  vmla_status s = check_compress_args(cfg, x, w_dkv_kr, cache);
+  if (s != VMLA_OK) return s;
   if (first_frame != cache->frames_written)
     return fail(VMLA_ERR_INVALID_ARG, "first_frame %lld does not follow frames_written %lld",
                 (long long)first_frame, (long long)cache->frames_written);
-  const FrameGeom g = make_geom(*cfg, first_frame);
-  const RopeTable rt = make_rope_table(*cfg);
-  cudaError_t e;
-  if (cfg->dtype == VMLA_F32) {
-    e = simt_compress_append<float>(*cfg, cache->batch, (const float*)x, (const float*)w_dkv_kr, g,
-                                    rt, (float*)cache->c, (float*)cache->k_r, as_stream(stream));
-  } else {
-    s = tc_check_compress(*cfg);
-    if (s != VMLA_OK) return fail(s, "%s", tc_last_reason());
-    e = tc_compress_append(*cfg, cache->batch, x, w_dkv_kr, g, rt, cache->c, cache->k_r,
-                           as_stream(stream));
-  }
-  if (e != cudaSuccess) return cuda_fail(e, "compress_append launch");
+  s = compress_chunk(cfg, x, w_dkv_kr, first_frame, cache, stream);
+  if (s != VMLA_OK) return s;
   cache->frames_written += cfg->chunk_frames;
   return VMLA_OK;
+}
+
+vmla_status vmla_compress_rewrite(const vmla_config* cfg, const void* x, const void* w_dkv_kr,
+                                  vmla_cache* cache, void* stream) {
+  vmla_status s = check_compress_args(cfg, x, w_dkv_kr, cache);
+  if (s != VMLA_OK) return s;
+  if (cache->frames_written < cfg->chunk_frames)
+    return fail(VMLA_ERR_INVALID_ARG, "no chunk to rewrite: frames_written %lld < chunk_frames %d",
+                (long long)cache->frames_written, cfg->chunk_frames);
+  return compress_chunk(cfg, x, w_dkv_kr, cache->frames_written - cfg->chunk_frames, cache, stream);
 }
 
 vmla_status vmla_absorb_q(const vmla_config* cfg, int32_t batch, int32_t n_query_chunks,
@@ -316,8 +380,10 @@ vmla_status vmla_rope_q(const vmla_config* cfg, int32_t batch, int32_t n_query_c
   return VMLA_OK;
 }
 
-vmla_status vmla_dense_append(const vmla_config* cfg, const void* x, const void* w_kv,
-                              int64_t first_frame, vmla_dense_cache* cache, void* stream) {
+namespace {
+
+vmla_status check_dense_append_args(const vmla_config* cfg, const void* x, const void* w_kv,
+                                    const vmla_dense_cache* cache) {
   vmla_status s = check_config(cfg);
   if (s != VMLA_OK) return s;
   if (!cache) return fail(VMLA_ERR_INVALID_ARG, "cache is NULL");
@@ -326,9 +392,11 @@ vmla_status vmla_dense_append(const vmla_config* cfg, const void* x, const void*
   VMLA_CHECK_PTR(cache->k);
   VMLA_CHECK_PTR(cache->v);
   if (cache->batch <= 0) return fail(VMLA_ERR_INVALID_ARG, "cache->batch must be >= 1");
-  if (first_frame != cache->frames_written)
-    return fail(VMLA_ERR_INVALID_ARG, "first_frame %lld does not follow frames_written %lld",
-                (long long)first_frame, (long long)cache->frames_written);
+  return VMLA_OK;
+}
+
+vmla_status dense_chunk(const vmla_config* cfg, const void* x, const void* w_kv, int64_t first_frame,
+                        vmla_dense_cache* cache, void* stream) {
   const FrameGeom g = make_geom(*cfg, first_frame);
   const RopeTable rt = make_rope_table(*cfg);
   cudaError_t e;
@@ -336,13 +404,37 @@ vmla_status vmla_dense_append(const vmla_config* cfg, const void* x, const void*
     e = simt_dense_append<float>(*cfg, cache->batch, (const float*)x, (const float*)w_kv, g, rt,
                                  (float*)cache->k, (float*)cache->v, as_stream(stream));
   } else {
-    s = tc_check_dense_append(*cfg);
+    vmla_status s = tc_check_dense_append(*cfg);
     if (s != VMLA_OK) return fail(s, "%s", tc_last_reason());
     e = tc_dense_append(*cfg, cache->batch, x, w_kv, g, rt, cache->k, cache->v, as_stream(stream));
   }
-  if (e != cudaSuccess) return cuda_fail(e, "dense_append launch");
+  if (e != cudaSuccess) return cuda_fail(e, "dense projection launch");
+  return VMLA_OK;
+}
+
+}  // namespace
+
+vmla_status vmla_dense_append(const vmla_config* cfg, const void* x, const void* w_kv,
+                              int64_t first_frame, vmla_dense_cache* cache, void* stream) {
+  vmla_status s = check_dense_append_args(cfg, x, w_kv, cache);
+  if (s != VMLA_OK) return s;
+  if (first_frame != cache->frames_written)
+    return fail(VMLA_ERR_INVALID_ARG, "first_frame %lld does not follow frames_written %lld",
+                (long long)first_frame, (long long)cache->frames_written);
+  s = dense_chunk(cfg, x, w_kv, first_frame, cache, stream);
+  if (s != VMLA_OK) return s;
   cache->frames_written += cfg->chunk_frames;
   return VMLA_OK;
+}
+
+vmla_status vmla_dense_rewrite(const vmla_config* cfg, const void* x, const void* w_kv,
+                               vmla_dense_cache* cache, void* stream) {
+  vmla_status s = check_dense_append_args(cfg, x, w_kv, cache);
+  if (s != VMLA_OK) return s;
+  if (cache->frames_written < cfg->chunk_frames)
+    return fail(VMLA_ERR_INVALID_ARG, "no chunk to rewrite: frames_written %lld < chunk_frames %d",
+                (long long)cache->frames_written, cfg->chunk_frames);
+  return dense_chunk(cfg, x, w_kv, cache->frames_written - cfg->chunk_frames, cache, stream);
 }
 
 vmla_status vmla_dense_mha(const vmla_config* cfg, const void* q, const vmla_dense_cache* cache,

@@ -23,7 +23,8 @@ EXPORTED = ("vmla_compress_append", "vmla_absorb_q", "vmla_latent_attention", "v
             "vmla_rope_q", "vmla_dense_append", "vmla_dense_mha", "vmla_device_status",
             "vmla_check_attention_window", "vmla_set_wait_timeout_ms", "vmla_debug_drop_kv_tile",
             "vmla_latent_cache_bytes", "vmla_dense_cache_bytes", "vmla_launch_count",
-            "vmla_status_string", "vmla_last_error_detail", "vmla_abi_version")
+            "vmla_status_string", "vmla_last_error_detail", "vmla_abi_version",
+            "vmla_compress_rewrite", "vmla_dense_rewrite", "vmla_plan_capacity")
 
 
 class VmlaError(RuntimeError):
@@ -44,6 +45,11 @@ class CConfig(ctypes.Structure):
 class CCache(ctypes.Structure):
     _fields_ = [("c", ctypes.c_void_p), ("k_r", ctypes.c_void_p), ("batch", ctypes.c_int32),
                 ("reserved", ctypes.c_int32), ("frames_written", ctypes.c_int64)]
+
+
+class CCapacity(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("max_batch", "cache_bytes_per_seq",
+                                                "buffer_bytes_per_seq", "weight_bytes")]
 
 
 class CDenseCache(ctypes.Structure):
@@ -68,6 +74,9 @@ def _load():
         "vmla_dense_mha": [cfgp, VP, P(CDenseCache), I64, I32, VP, VP, VP],
         "vmla_device_status": [VP, P(I32)],
         "vmla_check_attention_window": [cfgp, I64, I64, I32],
+        "vmla_compress_rewrite": [cfgp, VP, VP, P(CCache), VP],
+        "vmla_dense_rewrite": [cfgp, VP, VP, P(CDenseCache), VP],
+        "vmla_plan_capacity": [cfgp, I32, I32, I64, I64, I64, P(CCapacity)],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -188,6 +197,17 @@ def compress_append(cfg: VmlaConfig, x: torch.Tensor, w_dkv_kr: torch.Tensor, ca
                                    ff, ctypes.byref(cache.struct), _stream(x)))
 
 
+def compress_rewrite(cfg: VmlaConfig, x: torch.Tensor, w_dkv_kr: torch.Tensor,
+                     cache: LatentCache) -> None:
+    """Recompute the newest chunk's cache rows in place from x [B, F*T_f, D] (one denoising step of a
+    few-step chunk); frames_written is unchanged."""
+    B = cache.batch
+    cc = c_config(cfg)
+    check(LIB.vmla_compress_rewrite(ctypes.byref(cc), _arg(x, cfg, (B, cfg.chunk_tokens, cfg.dim), "x"),
+                                    _arg(w_dkv_kr, cfg, (cfg.d_c + cfg.d_rope, cfg.dim), "w_dkv_kr"),
+                                    ctypes.byref(cache.struct), _stream(x)))
+
+
 def absorb_q(cfg: VmlaConfig, q_nope: torch.Tensor, q_rope: torch.Tensor, w_uk: torch.Tensor,
              first_frame: int, n_query_chunks: int = 1, out: Optional[torch.Tensor] = None):
     B, nq = q_nope.shape[0], q_nope.shape[1]
@@ -261,6 +281,15 @@ def dense_append(cfg: VmlaConfig, x: torch.Tensor, w_kv: torch.Tensor, cache: De
                                 ff, ctypes.byref(cache.struct), _stream(x)))
 
 
+def dense_rewrite(cfg: VmlaConfig, x: torch.Tensor, w_kv: torch.Tensor, cache: DenseCache) -> None:
+    """Dense counterpart of compress_rewrite."""
+    B = cache.struct.batch
+    cc = c_config(cfg)
+    check(LIB.vmla_dense_rewrite(ctypes.byref(cc), _arg(x, cfg, (B, cfg.chunk_tokens, cfg.dim), "x"),
+                                 _arg(w_kv, cfg, (cfg.n_heads * (cfg.d_h + cfg.d_v), cfg.dim), "w_kv"),
+                                 ctypes.byref(cache.struct), _stream(x)))
+
+
 def dense_mha(cfg: VmlaConfig, q: torch.Tensor, cache: DenseCache, first_frame: int,
               n_query_chunks: int = 1, out: Optional[torch.Tensor] = None,
               lse: Optional[torch.Tensor] = None, want_lse: bool = False):
@@ -319,6 +348,17 @@ def dense_cache_bytes(cfg: VmlaConfig, batch: int) -> int:
     return int(LIB.vmla_dense_cache_bytes(ctypes.byref(cc), batch))
 
 
+def plan_capacity(cfg: VmlaConfig, n_layers: int, budget_bytes: int, *, dense: bool = False,
+                  fixed_bytes: int = 0, extra_bytes_per_seq: int = 0) -> dict:
+    """Largest batch of sequences whose n_layers caches, one layer step's tensors and the given extra
+    bytes fit ``budget_bytes`` (host-only; see vmla_plan_capacity)."""
+    cc = c_config(cfg)
+    out = CCapacity()
+    check(LIB.vmla_plan_capacity(ctypes.byref(cc), n_layers, 1 if dense else 0, int(budget_bytes),
+                                 int(fixed_bytes), int(extra_bytes_per_seq), ctypes.byref(out)))
+    return {n: int(getattr(out, n)) for n, _ in CCapacity._fields_}
+
+
 def layer_step(cfg: VmlaConfig, x: torch.Tensor, q_nope: torch.Tensor, q_rope: torch.Tensor,
                w_dkv_kr: torch.Tensor, w_uk: torch.Tensor, w_uv: torch.Tensor, cache: LatentCache,
                bufs: Optional[dict] = None) -> torch.Tensor:
@@ -336,4 +376,5 @@ def layer_step(cfg: VmlaConfig, x: torch.Tensor, q_nope: torch.Tensor, q_rope: t
 __all__ = ["LIB", "VmlaError", "LatentCache", "DenseCache", "compress_append", "absorb_q",
            "latent_attention", "value_up", "rope_q", "dense_append", "dense_mha", "device_status",
            "launch_count", "latent_cache_bytes", "dense_cache_bytes", "layer_step", "c_config",
+           "compress_rewrite", "dense_rewrite", "plan_capacity", "CCapacity",
            "CConfig", "CCache", "CDenseCache", "EXPORTED", "VMLA_F32", "VMLA_BF16"]

@@ -81,6 +81,16 @@ class OracleLayer:
             self.hist[b].append(c, k_r, pos[:, 0])
         self.frames_written += cfg.chunk_frames
 
+    def rewrite(self, x: torch.Tensor):
+        """Replace the newest chunk's entries with those computed from x (one denoising step)."""
+        cfg = self.cfg
+        f0 = self.frames_written - cfg.chunk_frames
+        pos = O.token_positions(f0, cfg.chunk_tokens, cfg.grid_h, cfg.grid_w)
+        xs = f64(x)
+        for b in range(self.batch):
+            c, k_r = O.compress(xs[b], self.w, cfg.d_c, pos, pairs(cfg), cfg.rope_theta)
+            self.hist[b].rewrite_newest(c, k_r, pos[:, 0])
+
     def ring(self, b: int):
         cfg = self.cfg
         c, written = O.ring_from_history(self.hist[b].c, self.frames_written, cfg.window_frames,
