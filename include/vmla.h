@@ -137,6 +137,22 @@ VMLA_API vmla_status vmla_latent_attention(const vmla_config* cfg, const void* q
                                   int64_t first_frame, int32_t n_query_chunks, void* out_latent,
                                   float* lse, void* stream);
 
+/* The three steps above in one launch: absorbed query, latent attention and value up-projection, with
+ * q_abs and the latent output kept on chip (same arithmetic and roundings as vmla_absorb_q ->
+ * vmla_latent_attention -> vmla_value_up: q~ and the latent output are rounded to bf16 before their
+ * next product).  VideoMLA technical summary, Method item 2 (per-head keys and values rebuilt from the
+ * shared latent by W^K_up,h and W^V_up,h) and item 3 (the rotated query part).
+ *   q_nope [batch, Nq, n_heads, d_nope], q_rope [batch, Nq, n_heads, d_rope],
+ *   w_uk [n_heads, d_nope, d_c], w_uv [n_heads, d_v, d_c]
+ *   -> out [batch, Nq, n_heads, d_v], lse [batch, Nq, n_heads] (natural log, or NULL).
+ * Same window rules as vmla_latent_attention.  bf16 only; needs d_rope == 32, d_c in {128, 192, 256},
+ * d_nope a multiple of 16 in [16, 128] and d_v a multiple of 32 in [32, 128] (VMLA_ERR_UNSUPPORTED
+ * otherwise). */
+VMLA_API vmla_status vmla_latent_attention_fused(const vmla_config* cfg, const void* q_nope, const void* q_rope,
+                                                 const void* w_uk, const void* w_uv, const vmla_cache* cache,
+                                                 int64_t first_frame, int32_t n_query_chunks, void* out,
+                                                 float* lse, void* stream);
+
 /* Value up-projection applied once to the attention-weighted latent (VideoMLA, Method item 2):
  *   out[b, n, h, :] = W^V_up,h out_latent[b, n, h, :]
  *   out_latent [batch, n_tokens, n_heads, d_c], w_uv [n_heads, d_v, d_c], out [batch, n_tokens, n_heads, d_v]. */

@@ -20,6 +20,16 @@
 // memory bandwidth and the tensor pipe stalls.  The TMEM budget (512 columns: 2 S buffers, O, Q) then
 // sets BN: 96 keys for d_c = 192, 128 keys for smaller latents and for the dense layer.
 // The KV ring is released by tcgen05.commit after the P V MMAs that last read a stage.
+//
+// The fused latent instance also does the two per-head projections around the attention (the
+// technical summary's Method item 2: keys and values are rebuilt from the latent with the per-head
+// up-projections).  Its tiles are 128 tokens of one head.  Prologue: q^nope (TMA, into the Q buffer) times
+// W^K_up,h (TMA, into the last KV stage) on the tensor cores gives q~ in the TMEM O columns; the
+// softmax warps round it to bf16 and write it, with RoPE3D(q^rope), into the Q buffer as the 128-byte /
+// 64-byte swizzled K-major operand that TMA would have produced.  Epilogue: O / l (bf16) goes back into
+// the Q buffer, W^V_up,h comes through the KV ring as one more "tile", and one MMA chain writes
+// o = (O / l) W^V_up,h^T into the first S buffer, from which the softmax warps store it.  q_abs and the
+// latent output never touch global memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -45,6 +55,24 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #endif
 constexpr int kPolyPairs = VMLA_EXP2_POLY_PAIRS;
 
+// Rotation of query pair p for the fused prologue: the angle is formed and reduced to [-pi, pi] in
+// double precision (large frame indices lose nothing), then the MUFU sine / cosine (absolute error
+// about 1e-6 on that interval, far below the bf16 rounding of the result) keep this once-per-row
+// step short.
+__device__ __forceinline__ void rope_rotate_mufu(const RopeTable& rt, int p, int64_t f, int64_t i, int64_t j,
+                                                 float a, float b, float* ra, float* rb) {
+  const int ax = rt.axis[p];
+  const double pos = (double)(ax == 0 ? f : (ax == 1 ? i : j));
+  const double two_pi = 6.283185307179586476925286766559;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
+  double ang = pos * rt.inv_freq[p];
+  ang = fma(-two_pi, rint(ang * inv_two_pi), ang);
+  float sf, cf;
+  __sincosf((float)ang, &sf, &cf);
+  *ra = a * cf - b * sf;
+  *rb = a * sf + b * cf;
+}
+
 struct AttnParams {
   const void* q;         // query rows (used when Q is kept in TMEM)
   int rows_per_b;        // query rows per batch element (latent: Nq*H, dense: Nq)
@@ -52,6 +80,7 @@ struct AttnParams {
   int heads;             // dense: heads per token (tile groups are (b, h)); latent: n = row / heads
   int dense;             // 1 for the per-head dense layer
   int64_t nq;            // query tokens per batch element
+  int head_major;        // tiles are 128 tokens of one head (dense and fused layers)
   FrameGeom g;
   float scale_log2;      // softmax_scale * log2(e)
   void* out;
@@ -59,6 +88,11 @@ struct AttnParams {
   int* status;
   uint64_t limit_ns;
   int drop_kv_tile;      // test hook: this KV tile is never loaded (-1: none)
+  // fused latent layer only
+  const void* q_rope;    // [B, Nq, H, 32] bf16: rotated in the prologue
+  int d_nope;            // K of the absorbing MMA (multiple of 16, <= 128)
+  int d_v;               // N of the value up-projection MMA (multiple of 32, <= BN)
+  RopeTable rt;          // 3D-RoPE pairs of the query rotation
 };
 
 // Compile-time plan of one kernel instance.
@@ -69,7 +103,7 @@ struct AttnParams {
 //   Q_TMEM  whether Q lives in TMEM (the A operand of S = Q K^T) or in shared memory
 //   ONES  V is extended by 16 columns of ones in shared memory, so that the P V MMA also produces
 //         the row sum of P in O's column DV (the softmax then needs no add chains)
-template <int KB, int KR, int VB, bool V_ALIAS, int BN, int NS, bool Q_TMEM, bool ONES>
+template <int KB, int KR, int VB, bool V_ALIAS, int BN, int NS, bool Q_TMEM, bool ONES, bool FUSED>
 struct Plan {
   static constexpr int kDQK = 64 * KB + KR;
   static constexpr int kDV = 64 * VB;
@@ -98,14 +132,19 @@ struct Plan {
   static_assert(kDV % 32 == 0 && (kDQK / 2) % 8 == 0, "row chunks");
   static_assert(!ONES || Q_TMEM, "the ones box is filled by the warps that also write Q into TMEM");
   static_assert(kNPV <= 256 && kNPV % 16 == 0, "P V MMA shape");
+  // fused: q^nope (two 64-column boxes) and then O / l must fit the Q buffer
+  static_assert(!FUSED || (!Q_TMEM && V_ALIAS && KR == 32 && !ONES && KB >= 2 &&
+                           kQBytes >= 2 * kBlockM * 128 && kQBytes >= VB * kBlockM * 128),
+                "fused layout");
 };
 
-template <int KB, int KR, int VB, bool V_ALIAS, int BN, int NS, bool Q_TMEM, bool ONES>
+template <int KB, int KR, int VB, bool V_ALIAS, int BN, int NS, bool Q_TMEM, bool ONES, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
 attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_qr,
                  const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_kr,
-                 const __grid_constant__ CUtensorMap map_v, const AttnParams p) {
-  using PL = Plan<KB, KR, VB, V_ALIAS, BN, NS, Q_TMEM, ONES>;
+                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_wuk,
+                 const __grid_constant__ CUtensorMap map_wuv, const AttnParams p) {
+  using PL = Plan<KB, KR, VB, V_ALIAS, BN, NS, Q_TMEM, ONES, FUSED>;
   constexpr int NST = PL::kStages;
   constexpr int DV = PL::kDV;
   constexpr int DQK = PL::kDQK;
@@ -121,7 +160,11 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   uint64_t* p_ready = s_full + NS;        // [NS][2]: P of the first / second half of the tile's keys
   uint64_t* pv_done = p_ready + 2 * NS;   // NS: P V of a tile of that S buffer completed
   uint64_t* drain = pv_done + NS;         // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* bar_pro = drain + 1;          // fused: q^nope and W^K_up,h landed
+  uint64_t* qa_full = bar_pro + 1;        // fused: q~ = q^nope W^K_up,h complete in TMEM
+  uint64_t* o_ready = qa_full + 1;        // fused: O / l written to shared memory (128 arrivals)
+  uint64_t* out_full = o_ready + 1;       // fused: the value up-projection complete in TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(out_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32;
@@ -130,16 +173,17 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   const int tile = blockIdx.x;
   const int group = tile / p.tiles_per_group;
   const int row0 = (tile % p.tiles_per_group) * kBlockM;      // first query row of the tile
-  const int b = p.dense ? group / p.heads : group;
-  const int h = p.dense ? group % p.heads : 0;
-  const int tok_div = p.dense ? 1 : p.heads;                   // query row -> token
+  const int b = p.head_major ? group / p.heads : group;
+  const int h = p.head_major ? group % p.heads : 0;
+  const int kv_h = p.dense ? h : 0;                            // head coordinate of the KV maps
+  const int tok_div = p.head_major ? 1 : p.heads;              // query row -> token
   const int last_row = min(row0 + kBlockM, p.rows_per_b) - 1;
   const int64_t kend_first = key_end_rows(p.g, row0 / tok_div);
   const int64_t kend_last = key_end_rows(p.g, last_row / tok_div);
   const int n_kv = (int)((kend_last + BN - 1) / BN);
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, Q_TMEM ? 128 : 1);
+    mbar_init(bar_q, (Q_TMEM || FUSED) ? 128 : 1);
     for (int s = 0; s < NST; ++s) { mbar_init(kv_full + s, 1); mbar_init(kv_empty + s, 1); }
     for (int s = 0; s < NS; ++s) {
       mbar_init(s_full + s, 1);
@@ -148,6 +192,10 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       mbar_init(pv_done + s, 1);
     }
     mbar_init(drain, 1);
+    mbar_init(bar_pro, 1);
+    mbar_init(qa_full, 1);
+    mbar_init(o_ready, 128);
+    mbar_init(out_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -166,30 +214,57 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     if (elect_one()) {
       tma_prefetch_desc(&map_k);
       if (!V_ALIAS) tma_prefetch_desc(&map_v);
-      if (!Q_TMEM) {
+      if (!Q_TMEM && !FUSED) {
         mbar_arrive_expect_tx(bar_q, PL::kQBytes);
         for (int i = 0; i < KB; ++i) tma_load_4d(sQ + i * kBlockM * 128, &map_q, bar_q, 64 * i, h, row0, b);
         if (KR) tma_load_4d(sQ + KB * kBlockM * 128, &map_qr, bar_q, 64 * KB, h, row0, b);
       }
+      if (FUSED) {
+        // prologue operands: the q^nope tile (two 64-column boxes; columns past d_nope read as zeros)
+        // into the Q buffer, W^K_up,h (d_c/64 boxes of [d_nope rows][64 columns]) into the last stage
+        tma_prefetch_desc(&map_wuk);
+        tma_prefetch_desc(&map_wuv);
+        uint8_t* wst = sKV + (NST - 1) * PL::kStageBytes;
+        mbar_arrive_expect_tx(bar_pro, 2 * kBlockM * 128 + VB * p.d_nope * 128);
+        for (int i = 0; i < 2; ++i) tma_load_4d(sQ + i * kBlockM * 128, &map_q, bar_pro, 64 * i, h, row0, b);
+        for (int i = 0; i < VB; ++i) tma_load_4d(wst + i * p.d_nope * 128, &map_wuk, bar_pro, 64 * i, 0, h, 0);
+      }
+      // load j goes to stage j % NST once the P V of load j - NST has completed; in the fused layer the
+      // last stage first holds W^K_up,h until the prologue MMA has completed
+      auto claim = [&](int j) -> bool {
+        const int st = j % NST;
+        if (j >= NST && !mbar_wait(kv_empty + st, ((j / NST) - 1) & 1, abort_flag, p.status, 1, p.limit_ns))
+          return false;
+        if (FUSED && j == NST - 1 && !mbar_wait(qa_full, 0, abort_flag, p.status, 8, p.limit_ns)) return false;
+        return true;
+      };
       int issued = 0;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % NST;
-        if (j >= NST && !mbar_wait(kv_empty + st, ((j / NST) - 1) & 1, abort_flag, p.status, 1, p.limit_ns))
-          break;
+        if (!claim(j)) break;
         issued = j + 1;
         if (j == p.drop_kv_tile) continue;
         uint8_t* stage = sKV + st * PL::kStageBytes;
         mbar_arrive_expect_tx(kv_full + st, PL::kLoadBytes);
         const int krow = j * BN;
-        for (int i = 0; i < KB; ++i) tma_load_4d(stage + i * PL::kBox, &map_k, kv_full + st, 64 * i, h, krow, b);
+        for (int i = 0; i < KB; ++i) tma_load_4d(stage + i * PL::kBox, &map_k, kv_full + st, 64 * i, kv_h, krow, b);
         if (KR) tma_load_4d(stage + PL::kRopeOff, &map_kr, kv_full + st, 0, 0, krow, b);
         if (!V_ALIAS)
           for (int i = 0; i < VB; ++i)
-            tma_load_4d(stage + PL::kVOff + i * PL::kBox, &map_v, kv_full + st, 64 * i, h, krow, b);
+            tma_load_4d(stage + PL::kVOff + i * PL::kBox, &map_v, kv_full + st, 64 * i, kv_h, krow, b);
+      }
+      if (FUSED && issued == n_kv && claim(n_kv)) {
+        // W^V_up,h (d_c/64 K-major boxes of [d_v rows][64 columns]) as load n_kv of the ring
+        const int st = n_kv % NST;
+        uint8_t* stage = sKV + st * PL::kStageBytes;
+        mbar_arrive_expect_tx(kv_full + st, VB * p.d_v * 128);
+        for (int i = 0; i < VB; ++i) tma_load_4d(stage + i * p.d_v * 128, &map_wuv, kv_full + st, 64 * i, 0, h, 0);
+        issued = n_kv + 1;
       }
       if (*abort_flag) {
         // let the copies already issued land before the CTA exits
-        if (!Q_TMEM) mbar_wait(bar_q, 0, &zero_flag, nullptr, 0, p.limit_ns);
+        if (!Q_TMEM && !FUSED) mbar_wait(bar_q, 0, &zero_flag, nullptr, 0, p.limit_ns);
+        if (FUSED) mbar_wait(bar_pro, 0, &zero_flag, nullptr, 0, p.limit_ns);
         for (int j = (issued > NST ? issued - NST : 0); j < issued; ++j)
           if (j != p.drop_kv_tile) mbar_wait(kv_full + j % NST, (j / NST) & 1, &zero_flag, nullptr, 0, p.limit_ns);
       }
@@ -201,7 +276,24 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, PL::kNPV, 0, 1);
       const uint32_t q_base = smem_u32(sQ);
       const uint32_t kv_base = smem_u32(sKV);
-      bool ok = mbar_wait(bar_q, 0, abort_flag, p.status, 2, p.limit_ns);
+      bool ok = true;
+      if (FUSED) {
+        ok = mbar_wait(bar_pro, 0, abort_flag, p.status, 9, p.limit_ns);
+        if (ok) {
+          tc_fence_after();
+          // q~ = q^nope W^K_up,h into the O columns: A K-major (two 64-column boxes), B MN-major
+          // ([d_nope rows][64 columns] boxes d_nope*128 B apart = LBO; a K step of 16 rows is 2048 B)
+          const uint32_t w_base = kv_base + (NST - 1) * PL::kStageBytes;
+          const uint32_t idesc_qa = idesc_bf16_f32(kBlockM, DV, 0, 1);
+          for (int k = 0; k < p.d_nope / 16; ++k) {
+            const uint64_t adesc = smem_desc(q_base + (k >> 2) * kBlockM * 128 + (k & 3) * 32, 16, 1024, kSwizzle128B);
+            const uint64_t bdesc = smem_desc(w_base + k * 2048, p.d_nope * 128, 1024, kSwizzle128B);
+            mma_ss(tmem + PL::kTmemO, adesc, bdesc, idesc_qa, k > 0 ? 1u : 0u);
+          }
+          mma_commit(qa_full);
+        }
+      }
+      ok = ok && mbar_wait(bar_q, 0, abort_flag, p.status, 2, p.limit_ns);
       // P V of tile jp in two halves of the keys: the first half's MMAs run while the softmax warps
       // still produce the second half's P
       auto issue_pv = [&](int jp) -> bool {
@@ -262,7 +354,29 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       // every MMA of this CTA has completed before TMEM is released; the softmax warps also wait
       // on this single-phase barrier for the final O
       mma_commit(drain);
-      mbar_wait(drain, 0, &zero_flag, nullptr, 0, p.limit_ns);
+      if (FUSED) {
+        if (ok) {
+          const int st = n_kv % NST;
+          ok = mbar_wait(kv_full + st, (n_kv / NST) & 1, abort_flag, p.status, 10, p.limit_ns) &&
+               mbar_wait(o_ready, 0, abort_flag, p.status, 11, p.limit_ns);
+          if (ok) {
+            tc_fence_after();
+            // o = (O / l) W^V_up,h^T into the first S buffer: A = O / l (bf16 K-major boxes in the Q
+            // buffer, written after every earlier MMA completed), B = W^V_up,h (K-major boxes)
+            const uint32_t wv = kv_base + st * PL::kStageBytes;
+            const uint32_t idesc_vu = idesc_bf16_f32(kBlockM, p.d_v, 0, 0);
+            for (int k = 0; k < DV / 16; ++k) {
+              const uint64_t adesc = smem_desc(q_base + (k >> 2) * kBlockM * 128 + (k & 3) * 32, 16, 1024, kSwizzle128B);
+              const uint64_t bdesc = smem_desc(wv + (k >> 2) * p.d_v * 128 + (k & 3) * 32, 16, 1024, kSwizzle128B);
+              mma_ss(tmem, adesc, bdesc, idesc_vu, k > 0 ? 1u : 0u);
+            }
+          }
+        }
+        mma_commit(out_full);
+        mbar_wait(out_full, 0, &zero_flag, nullptr, 0, p.limit_ns);
+      } else {
+        mbar_wait(drain, 0, &zero_flag, nullptr, 0, p.limit_ns);
+      }
     }
   } else {
     // ========= query rows, softmax, epilogue (warps 0-3; thread = query row = TMEM lane) =========
@@ -272,7 +386,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const int64_t kend = row_valid ? key_end_rows(p.g, row / tok_div) : kend_last;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     int64_t orow;                                   // this row's index in [rows of q / out / lse]
-    if (p.dense) orow = (((int64_t)b * p.nq + row) * p.heads + h);
+    if (p.head_major) orow = (((int64_t)b * p.nq + row) * p.heads + h);
     else orow = (int64_t)b * p.rows_per_b + row;
 
     if (Q_TMEM) {
@@ -308,6 +422,73 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
     float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = true;
+    if (FUSED) {
+      // the Q row, written as the K-major operand TMA would have produced (16-byte chunk k of a
+      // 128-byte row of a c box at chunk k ^ (row % 8); of a 64-byte rope row at chunk k ^ ((row / 2) % 4)).
+      // First RoPE3D(q^rope) of the row's token into the rope box, which the prologue's TMA copies do not
+      // touch, while the q^nope W^K_up,h MMA is still in flight; then q~ (fp32, O columns) as bf16.
+      {
+        float v[32];
+        if (row_valid) {
+          const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.q_rope) + orow * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 u = src[q];
+            const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) v[8 * q + t] = __bfloat162float(e[t]);
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) v[t] = 0.f;
+        }
+        const int64_t f = p.g.first_frame + row / p.g.tokens_per_frame;
+        const int rr = row % p.g.tokens_per_frame;
+        const int ri = rr / p.g.grid_w, rj = rr % p.g.grid_w;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float a, bb;
+          rope_rotate_mufu(p.rt, q, f, ri, rj, v[2 * q], v[2 * q + 1], &a, &bb);
+          v[2 * q] = a;
+          v[2 * q + 1] = bb;
+        }
+        uint8_t* ropep = sQ + KB * (kBlockM * 128) + r * 64;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 w;
+          w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+          w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+          w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+          w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+          *reinterpret_cast<uint4*>(ropep + ((q ^ ((r >> 1) & 3)) << 4)) = w;
+        }
+      }
+      const bool got = mbar_wait(qa_full, 0, abort_flag, p.status, 12, p.limit_ns);
+      ok = __all_sync(0xffffffffu, got);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < DV / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + PL::kTmemO + c * 32, v);
+          tmem_ld_wait();
+          uint8_t* rowp = sQ + (c >> 1) * (kBlockM * 128) + r * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = (c & 1) * 4 + q;
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+            w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+            w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+            w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+            *reinterpret_cast<uint4*>(rowp + ((chunk ^ (r & 7)) << 4)) = w;
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar_q);
+      }
+    }
     // Wait until P_{j-1} V_{j-1} has completed: phase (j-1)/NS of pv_done[(j-1) % NS].  Called from tile
     // j, where that barrier is at most one phase away: s_full[j] completing implies that
     // P_{j-1-NS} V_{j-1-NS} completed (issued before S_j), and P_{j-1+NS} V_{j-1+NS} cannot start
@@ -318,7 +499,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       return __all_sync(0xffffffffu, got);
     };
     const float sc = p.scale_log2;
-    for (int j = 0; j < n_kv; ++j) {
+    for (int j = 0; ok && j < n_kv; ++j) {
       const int bj = j % NS;
       const bool got = mbar_wait(s_full + bj, (j / NS) & 1, abort_flag, p.status, 6, p.limit_ns);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -426,8 +607,52 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       }
       const float inv_l = 1.f / l_row;
       __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out);
+      if (FUSED) {
+        // O / l rounded to bf16 into the Q buffer (every S = Q K^T MMA has completed): the A operand
+        // of the value up-projection, same swizzled K-major layout as q~
 #pragma unroll
-      for (int c = 0; c < DV / 32; ++c) {
+        for (int c = 0; c < DV / 32; ++c) {
+          tmem_ld32(tmem + lane_base + PL::kTmemO + c * 32, o);
+          tmem_ld_wait();
+          uint8_t* rowp = sQ + (c >> 1) * (kBlockM * 128) + r * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = (c & 1) * 4 + q;
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(rowp + ((chunk ^ (r & 7)) << 4)) = v;
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(o_ready);
+        bool got = mbar_wait(out_full, 0, abort_flag, p.status, 13, p.limit_ns);
+        got = __all_sync(0xffffffffu, got && !*abort_flag);
+        if (got) {
+          tc_fence_after();
+          for (int c = 0; c < p.d_v / 32; ++c) {
+            tmem_ld32(tmem + lane_base + c * 32, o);
+            tmem_ld_wait();
+            if (row_valid) {
+              uint4* dst = reinterpret_cast<uint4*>(out + orow * p.d_v + c * 32);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(o[8 * q + 0]), __uint_as_float(o[8 * q + 1]));
+                v.y = pack_bf16x2(__uint_as_float(o[8 * q + 2]), __uint_as_float(o[8 * q + 3]));
+                v.z = pack_bf16x2(__uint_as_float(o[8 * q + 4]), __uint_as_float(o[8 * q + 5]));
+                v.w = pack_bf16x2(__uint_as_float(o[8 * q + 6]), __uint_as_float(o[8 * q + 7]));
+                dst[q] = v;
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < (FUSED ? 0 : DV / 32); ++c) {
         tmem_ld32(tmem + lane_base + PL::kTmemO + c * 32, o);
         tmem_ld_wait();
         if (row_valid) {
@@ -454,14 +679,14 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   }
 }
 
-template <int KB, int KR, int VB, bool V_ALIAS, int BN, int NS, bool Q_TMEM, bool ONES>
+template <int KB, int KR, int VB, bool V_ALIAS, int BN, int NS, bool Q_TMEM, bool ONES, bool FUSED>
 cudaError_t launch_attention(const TmaMaps5& m, const AttnParams& p, int n_tiles, cudaStream_t st) {
-  using PL = Plan<KB, KR, VB, V_ALIAS, BN, NS, Q_TMEM, ONES>;
-  auto kern = attention_kernel<KB, KR, VB, V_ALIAS, BN, NS, Q_TMEM, ONES>;
+  using PL = Plan<KB, KR, VB, V_ALIAS, BN, NS, Q_TMEM, ONES, FUSED>;
+  auto kern = attention_kernel<KB, KR, VB, V_ALIAS, BN, NS, Q_TMEM, ONES, FUSED>;
   static std::atomic<uint64_t> done{0};
   cudaError_t attr_err = ensure_smem_attr((const void*)kern, PL::kSmemBytes, done);
   if (attr_err != cudaSuccess) return attr_err;
-  kern<<<n_tiles, kThreads, PL::kSmemBytes, st>>>(m.q, m.qr, m.k, m.kr, m.v, p);
+  kern<<<n_tiles, kThreads, PL::kSmemBytes, st>>>(m.q, m.qr, m.k, m.kr, m.v, m.wuk, m.wuv, p);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -513,12 +738,15 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
   if ((e = make_map_4d(&m.kr, k_r, 32, 1, valid_rows, batch, 64, 64, cap * 64, 32, 1, kv_box_rows, 64)) != cudaSuccess)
     return e;
   m.v = m.k;
+  m.wuk = m.k;
+  m.wuv = m.k;
   AttnParams p{};
   p.q = q_abs;
   p.rows_per_b = (int)rows;
   p.tiles_per_group = (int)((rows + kBlockM - 1) / kBlockM);
   p.heads = H;
   p.dense = 0;
+  p.head_major = 0;
   p.nq = nq;
   p.g = g;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -529,10 +757,93 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
   p.drop_kv_tile = take_drop_kv_tile();
   const int n_tiles = batch * p.tiles_per_group;
   switch (cfg.d_c) {
-    case 64: return launch_attention<1, 32, 1, true, kLatentBN, 2, true, false>(m, p, n_tiles, st);
-    case 128: return launch_attention<2, 32, 2, true, kLatentBN, 2, true, false>(m, p, n_tiles, st);
-    case 192: return launch_attention<3, 32, 3, true, kLatentBN, 2, false, false>(m, p, n_tiles, st);
-    default: return launch_attention<4, 32, 4, true, kLatentBN, 2, false, false>(m, p, n_tiles, st);
+    case 64: return launch_attention<1, 32, 1, true, kLatentBN, 2, true, false, false>(m, p, n_tiles, st);
+    case 128: return launch_attention<2, 32, 2, true, kLatentBN, 2, true, false, false>(m, p, n_tiles, st);
+    case 192: return launch_attention<3, 32, 3, true, kLatentBN, 2, false, false, false>(m, p, n_tiles, st);
+    default: return launch_attention<4, 32, 4, true, kLatentBN, 2, false, false, false>(m, p, n_tiles, st);
+  }
+}
+
+namespace {
+
+// Fused instances: Q in shared memory (the prologue writes it there), 128-key tiles, two S buffers.
+template <int KB>
+using FusedPlan = Plan<KB, 32, KB, true, kLatentBN, 2, false, false, true>;
+
+template <int KB>
+bool fused_fits(int d_nope, int d_v) {
+  return KB * d_nope * 128 <= FusedPlan<KB>::kStageBytes && KB * d_v * 128 <= FusedPlan<KB>::kStageBytes;
+}
+
+}  // namespace
+
+vmla_status tc_check_fused_attention(const vmla_config& c) {
+  if (c.d_rope != 32) { set_tc_reason("fused latent attention needs d_rope == 32"); return VMLA_ERR_UNSUPPORTED; }
+  if (c.d_c != 128 && c.d_c != 192 && c.d_c != 256) {
+    set_tc_reason("fused latent attention needs d_c in {128, 192, 256}");
+    return VMLA_ERR_UNSUPPORTED;
+  }
+  if (c.d_nope % 16 || c.d_nope < 16 || c.d_nope > 128) {
+    set_tc_reason("fused latent attention needs d_nope a multiple of 16 in [16, 128]");
+    return VMLA_ERR_UNSUPPORTED;
+  }
+  if (c.d_v % 32 || c.d_v < 32 || c.d_v > kLatentBN) {
+    set_tc_reason("fused latent attention needs d_v a multiple of 32 in [32, 128]");
+    return VMLA_ERR_UNSUPPORTED;
+  }
+  const bool fits = c.d_c == 128 ? fused_fits<2>(c.d_nope, c.d_v)
+                    : c.d_c == 192 ? fused_fits<3>(c.d_nope, c.d_v) : fused_fits<4>(c.d_nope, c.d_v);
+  if (!fits) { set_tc_reason("fused latent attention: up-projection weights exceed a KV stage"); return VMLA_ERR_UNSUPPORTED; }
+  return VMLA_OK;
+}
+
+cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t nq, const void* q_nope,
+                                      const void* q_rope, const void* w_uk, const void* w_uv, const void* c,
+                                      const void* k_r, int64_t cap, int64_t valid_rows, const FrameGeom& g,
+                                      const RopeTable& rt, float scale, void* out, float* lse, int* status,
+                                      cudaStream_t st) {
+  const int H = cfg.n_heads, dn = cfg.d_nope, dc = cfg.d_c, dv = cfg.d_v;
+  TmaMaps5 m{};
+  cudaError_t e;
+  // q^nope [B, Nq, H, d_nope] as {d_nope, H, Nq, B}: a 128-token box of one head
+  if ((e = make_map_4d(&m.q, q_nope, dn, H, nq, batch, (int64_t)dn * 2, (int64_t)H * dn * 2,
+                       nq * H * dn * 2, 64, 1, kBlockM, 128)) != cudaSuccess) return e;
+  m.qr = m.q;
+  if ((e = make_map_4d(&m.k, c, dc, 1, valid_rows, batch, (int64_t)dc * 2, (int64_t)dc * 2,
+                       cap * dc * 2, 64, 1, kLatentBN, 128)) != cudaSuccess) return e;
+  if ((e = make_map_4d(&m.kr, k_r, 32, 1, valid_rows, batch, 64, 64, cap * 64, 32, 1, kLatentBN, 64)) != cudaSuccess)
+    return e;
+  m.v = m.k;
+  // W^K_up [H, d_nope, d_c] as {d_c, d_nope, H, 1}: [d_nope rows][64 columns] boxes (MN-major B)
+  if ((e = make_map_4d(&m.wuk, w_uk, dc, dn, H, 1, (int64_t)dc * 2, (int64_t)dn * dc * 2,
+                       (int64_t)H * dn * dc * 2, 64, dn, 1, 128)) != cudaSuccess) return e;
+  // W^V_up [H, d_v, d_c] as {d_c, d_v, H, 1}: [d_v rows][64 columns] boxes (K-major B)
+  if ((e = make_map_4d(&m.wuv, w_uv, dc, dv, H, 1, (int64_t)dc * 2, (int64_t)dv * dc * 2,
+                       (int64_t)H * dv * dc * 2, 64, dv, 1, 128)) != cudaSuccess) return e;
+  AttnParams p{};
+  p.q = q_nope;
+  p.rows_per_b = (int)nq;
+  p.tiles_per_group = (int)((nq + kBlockM - 1) / kBlockM);
+  p.heads = H;
+  p.dense = 0;
+  p.head_major = 1;
+  p.nq = nq;
+  p.g = g;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = out;
+  p.lse = lse;
+  p.status = status;
+  p.limit_ns = wait_limit_ns();
+  p.drop_kv_tile = -1;
+  p.q_rope = q_rope;
+  p.d_nope = dn;
+  p.d_v = dv;
+  p.rt = rt;
+  const int n_tiles = batch * H * p.tiles_per_group;
+  switch (dc) {
+    case 128: return launch_attention<2, 32, 2, true, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
+    case 192: return launch_attention<3, 32, 3, true, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
+    default: return launch_attention<4, 32, 4, true, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
   }
 }
 
@@ -552,12 +863,15 @@ cudaError_t tc_dense_mha(const vmla_config& cfg, int batch, int64_t nq, const vo
   m.kr = m.k;
   if ((e = make_map_4d(&m.v, v, D, H, valid_rows, batch, D * 2, (int64_t)H * D * 2, cap * H * D * 2, 64, 1,
                        kBN, 128)) != cudaSuccess) return e;
+  m.wuk = m.k;
+  m.wuv = m.k;
   AttnParams p{};
   p.q = q;
   p.rows_per_b = (int)nq;
   p.tiles_per_group = (int)((nq + kBlockM - 1) / kBlockM);
   p.heads = H;
   p.dense = 1;
+  p.head_major = 1;
   p.nq = nq;
   p.g = g;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -567,7 +881,7 @@ cudaError_t tc_dense_mha(const vmla_config& cfg, int batch, int64_t nq, const vo
   p.limit_ns = wait_limit_ns();
   p.drop_kv_tile = -1;
   const int n_tiles = batch * H * p.tiles_per_group;
-  return launch_attention<2, 0, 2, false, kBN, 2, true, false>(m, p, n_tiles, st);
+  return launch_attention<2, 0, 2, false, kBN, 2, true, false, false>(m, p, n_tiles, st);
 }
 
 }  // namespace vmla

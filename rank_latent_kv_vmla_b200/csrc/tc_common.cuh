@@ -12,6 +12,7 @@ namespace vmla {
 
 struct TmaMaps5 {
   CUtensorMap q, qr, k, kr, v;
+  CUtensorMap wuk, wuv;   // fused latent attention: W^K_up and W^V_up
 };
 
 // Encode a 4-D bf16 tensor map {d0 (contiguous), d1, d2, d3} with byte strides s1, s2, s3 of the

@@ -335,6 +335,42 @@ vmla_status vmla_latent_attention(const vmla_config* cfg, const void* q_abs, con
   return VMLA_OK;
 }
 
+vmla_status vmla_latent_attention_fused(const vmla_config* cfg, const void* q_nope, const void* q_rope,
+                                        const void* w_uk, const void* w_uv, const vmla_cache* cache,
+                                        int64_t first_frame, int32_t n_query_chunks, void* out, float* lse,
+                                        void* stream) {
+  vmla_status s = check_config(cfg);
+  if (s != VMLA_OK) return s;
+  if (!cache) return fail(VMLA_ERR_INVALID_ARG, "cache is NULL");
+  VMLA_CHECK_PTR(q_nope);
+  VMLA_CHECK_PTR(q_rope);
+  VMLA_CHECK_PTR(w_uk);
+  VMLA_CHECK_PTR(w_uv);
+  VMLA_CHECK_PTR(cache->c);
+  VMLA_CHECK_PTR(cache->k_r);
+  VMLA_CHECK_PTR(out);
+  if (lse && !aligned16(lse)) return fail(VMLA_ERR_MISALIGNED, "lse is not 16-byte aligned");
+  if (cache->batch <= 0) return fail(VMLA_ERR_INVALID_ARG, "cache->batch must be >= 1");
+  if (cfg->dtype != VMLA_BF16)
+    return fail(VMLA_ERR_UNSUPPORTED, "the fused call runs on the bf16 tensor-core path only");
+  s = check_window(*cfg, cache->frames_written, first_frame, n_query_chunks);
+  if (s != VMLA_OK) return s;
+  s = tc_check_fused_attention(*cfg);
+  if (s != VMLA_OK) return fail(s, "%s", tc_last_reason());
+  const FrameGeom g = make_geom(*cfg, first_frame);
+  const RopeTable rt = make_rope_table(*cfg);
+  const int64_t T_f = (int64_t)cfg->grid_h * cfg->grid_w;
+  const int64_t nq = (int64_t)n_query_chunks * cfg->chunk_frames * T_f;
+  const int64_t cap = (int64_t)cfg->window_frames * T_f;
+  const int64_t valid_rows =
+      (cache->frames_written < cfg->window_frames ? cache->frames_written : cfg->window_frames) * T_f;
+  cudaError_t e = tc_latent_attention_fused(*cfg, cache->batch, nq, q_nope, q_rope, w_uk, w_uv, cache->c,
+                                            cache->k_r, cap, valid_rows, g, rt, softmax_scale(*cfg), out,
+                                            lse, device_status_ptr(), as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "latent_attention_fused launch");
+  return VMLA_OK;
+}
+
 vmla_status vmla_value_up(const vmla_config* cfg, int32_t batch, int64_t n_tokens,
                           const void* out_latent, const void* w_uv, void* out, void* stream) {
   vmla_status s = check_config(cfg);

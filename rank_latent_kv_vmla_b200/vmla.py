@@ -24,7 +24,8 @@ EXPORTED = ("vmla_compress_append", "vmla_absorb_q", "vmla_latent_attention", "v
             "vmla_check_attention_window", "vmla_set_wait_timeout_ms", "vmla_debug_drop_kv_tile",
             "vmla_latent_cache_bytes", "vmla_dense_cache_bytes", "vmla_launch_count",
             "vmla_status_string", "vmla_last_error_detail", "vmla_abi_version",
-            "vmla_compress_rewrite", "vmla_dense_rewrite", "vmla_plan_capacity")
+            "vmla_compress_rewrite", "vmla_dense_rewrite", "vmla_plan_capacity",
+            "vmla_latent_attention_fused")
 
 
 class VmlaError(RuntimeError):
@@ -77,6 +78,7 @@ def _load():
         "vmla_compress_rewrite": [cfgp, VP, VP, P(CCache), VP],
         "vmla_dense_rewrite": [cfgp, VP, VP, P(CDenseCache), VP],
         "vmla_plan_capacity": [cfgp, I32, I32, I64, I64, I64, P(CCapacity)],
+        "vmla_latent_attention_fused": [cfgp, VP, VP, VP, VP, P(CCache), I64, I32, VP, VP, VP],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -246,6 +248,29 @@ def latent_attention(cfg: VmlaConfig, q_abs: torch.Tensor, cache: LatentCache, f
     return (out, lse) if (lse is not None) else out
 
 
+def latent_attention_fused(cfg: VmlaConfig, q_nope: torch.Tensor, q_rope: torch.Tensor, w_uk: torch.Tensor,
+                           w_uv: torch.Tensor, cache: LatentCache, first_frame: int, n_query_chunks: int = 1,
+                           out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                           want_lse: bool = False):
+    """Absorbed query + latent attention + value up-projection in one launch:
+    q^nope [B, Nq, H, d_nope], q^rope [B, Nq, H, d_rope] -> o [B, Nq, H, d_v] (and lse [B, Nq, H])."""
+    B, nq, H = cache.batch, q_nope.shape[1], cfg.n_heads
+    if out is None:
+        out = torch.empty((B, nq, H, cfg.d_v), dtype=_dtype(cfg), device=q_nope.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, nq, H), dtype=torch.float32, device=q_nope.device)
+    if nq != n_query_chunks * cfg.chunk_tokens:
+        raise ValueError("q_nope covers %d tokens, expected %d" % (nq, n_query_chunks * cfg.chunk_tokens))
+    cc = c_config(cfg)
+    check(LIB.vmla_latent_attention_fused(
+        ctypes.byref(cc), _arg(q_nope, cfg, (B, nq, H, cfg.d_nope), "q_nope"),
+        _arg(q_rope, cfg, (B, nq, H, cfg.d_rope), "q_rope"), _arg(w_uk, cfg, (H, cfg.d_nope, cfg.d_c), "w_uk"),
+        _arg(w_uv, cfg, (H, cfg.d_v, cfg.d_c), "w_uv"), ctypes.byref(cache.struct), first_frame, n_query_chunks,
+        _arg(out, cfg, (B, nq, H, cfg.d_v), "out"), lse.data_ptr() if lse is not None else None,
+        _stream(q_nope)))
+    return (out, lse) if (lse is not None) else out
+
+
 def value_up(cfg: VmlaConfig, o_latent: torch.Tensor, w_uv: torch.Tensor,
              out: Optional[torch.Tensor] = None):
     B, n, H = o_latent.shape[0], o_latent.shape[1], cfg.n_heads
@@ -376,5 +401,5 @@ def layer_step(cfg: VmlaConfig, x: torch.Tensor, q_nope: torch.Tensor, q_rope: t
 __all__ = ["LIB", "VmlaError", "LatentCache", "DenseCache", "compress_append", "absorb_q",
            "latent_attention", "value_up", "rope_q", "dense_append", "dense_mha", "device_status",
            "launch_count", "latent_cache_bytes", "dense_cache_bytes", "layer_step", "c_config",
-           "compress_rewrite", "dense_rewrite", "plan_capacity", "CCapacity",
+           "compress_rewrite", "dense_rewrite", "plan_capacity", "CCapacity", "latent_attention_fused",
            "CConfig", "CCache", "CDenseCache", "EXPORTED", "VMLA_F32", "VMLA_BF16"]

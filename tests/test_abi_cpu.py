@@ -168,3 +168,22 @@ def test_plan_capacity_rejects_bad_arguments():
         assert st == V.VMLA_ERR_INVALID_ARG
     st, _ = _status(V.LIB.vmla_plan_capacity, ctypes.byref(cc), 30, 0, 10, 0, 0, None)
     assert st == V.VMLA_ERR_INVALID_ARG
+
+
+def test_fused_attention_rejects_unsupported_shapes():
+    """The fused call refuses, before launching, the fp32 path and shapes outside its layout."""
+    cache = _cache(frames_written=TINY.chunk_frames)
+    for bad, why in ((TINY, "bf16"), (WAN.replace(d_c=64), "d_c"), (WAN.replace(d_nope=88, rope_pairs_t=6), "d_nope"),
+                     (WAN.replace(d_v=160), "d_v")):
+        cc = V.c_config(bad)
+        c = _cache(frames_written=bad.chunk_frames)
+        st, detail = _status(V.LIB.vmla_latent_attention_fused, ctypes.byref(cc), FAKE, FAKE, FAKE, FAKE,
+                             ctypes.byref(c), 0, 1, FAKE, None, None)
+        assert st == V.VMLA_ERR_UNSUPPORTED, (why, st, detail)
+    cc = V.c_config(WAN)
+    st, _ = _status(V.LIB.vmla_latent_attention_fused, ctypes.byref(cc), FAKE, FAKE, FAKE, FAKE,
+                    ctypes.byref(_cache(frames_written=0)), 0, 1, FAKE, None, None)
+    assert st == V.VMLA_ERR_INVALID_ARG                       # nothing appended yet
+    st, _ = _status(V.LIB.vmla_latent_attention_fused, ctypes.byref(cc), FAKE + 8, FAKE, FAKE, FAKE,
+                    ctypes.byref(_cache(frames_written=3)), 0, 1, FAKE, None, None)
+    assert st == V.VMLA_ERR_MISALIGNED
