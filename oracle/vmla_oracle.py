@@ -301,15 +301,19 @@ def layer_reference(hist: History, q_nope, q_rope, w_uk, w_uv, *, first_frame, q
 # ---------------------------------------------------------------------------------------------------
 # Batch capacity at a fixed memory budget  [TS-R], [TS-M4]
 # ---------------------------------------------------------------------------------------------------
-def step_tensors(batch: int, *, dim, n_heads, d_nope, d_rope, d_c, d_v, tokens_per_chunk, dense):
+def step_tensors(batch: int, *, dim, n_heads, d_nope, d_rope, d_c, d_v, tokens_per_chunk, dense,
+                 fused=False):
     """Shapes of the tensors one layer step holds for ``batch`` sequences (reused by every layer):
     the chunk features and, latent path, q^nope, q^rope, the absorbed query, the latent output and the
-    output; dense path, the query and the output."""
+    output (the fused latent step keeps the absorbed query and the latent output on chip); dense path,
+    the query and the output."""
     B, N, H = batch, tokens_per_chunk, n_heads
     if dense:
         return {"x": (B, N, dim), "q": (B, N, H, d_nope + d_rope), "out": (B, N, H, d_v)}
-    return {"x": (B, N, dim), "q_nope": (B, N, H, d_nope), "q_rope": (B, N, H, d_rope),
-            "q_abs": (B, N, H, d_c + d_rope), "out_latent": (B, N, H, d_c), "out": (B, N, H, d_v)}
+    t = {"x": (B, N, dim), "q_nope": (B, N, H, d_nope), "q_rope": (B, N, H, d_rope), "out": (B, N, H, d_v)}
+    if not fused:
+        t.update({"q_abs": (B, N, H, d_c + d_rope), "out_latent": (B, N, H, d_c)})
+    return t
 
 
 def layer_weights(*, dim, n_heads, d_nope, d_rope, d_c, d_v, dense):
@@ -321,7 +325,7 @@ def layer_weights(*, dim, n_heads, d_nope, d_rope, d_c, d_v, dense):
 
 
 def memory_bytes(batch: int, *, n_layers, window_tokens, elt_bytes, fixed_bytes, extra_bytes_per_seq,
-                 dense, **shape) -> int:
+                 dense, fused=False, **shape) -> int:
     """Every byte held at once for ``batch`` sequences: each layer's cache (per token the dense
     2*n_h*d_h or the latent d_c + d_rope scalars [TS-M4]), each layer's weights, one layer step's tensors,
     the caller's fixed bytes and its per-sequence extra bytes."""
@@ -332,7 +336,7 @@ def memory_bytes(batch: int, *, n_layers, window_tokens, elt_bytes, fixed_bytes,
     scalars = n_layers * batch * window_tokens * per_token
     scalars += n_layers * sum(int(np.prod(v)) for v in layer_weights(dense=dense, **{
         k: shape[k] for k in ("dim", "n_heads", "d_nope", "d_rope", "d_c", "d_v")}).values())
-    scalars += sum(int(np.prod(v)) for v in step_tensors(batch, dense=dense, **shape).values())
+    scalars += sum(int(np.prod(v)) for v in step_tensors(batch, dense=dense, fused=fused, **shape).values())
     return scalars * elt_bytes + fixed_bytes + batch * extra_bytes_per_seq
 
 
