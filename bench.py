@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--batch", type=int, default=1, help="sequences per GPU")
     ap.add_argument("--impl", default="vmla", choices=["vmla", "reference"])
     ap.add_argument("--no-dense", action="store_true", help="skip the dense MHA comparison arm")
+    ap.add_argument("--path", default="fused", choices=["fused", "three"],
+                    help="fused: compress + one fused attention launch per step; three: compress + "
+                         "absorb + attention + value-up launches (the other path is timed beside it)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--workload", default="layer", choices=["layer", "batch8", "dc_sweep", "rollout", "fewstep",
@@ -75,6 +78,12 @@ def kernel_bytes(cfg, batch):
         "absorb_q": batch * nq * H * (cfg.d_nope + cfg.d_rope + cfg.d_qk) * e + H * cfg.d_nope * cfg.d_c * e,
         "value_up": batch * nq * H * (cfg.d_c + cfg.d_v) * e + H * cfg.d_v * cfg.d_c * e,
     }
+
+
+def projection_flops(cfg, batch) -> float:
+    """Flops of the two per-head projections the fused kernel also performs:
+    2*B*Nq*H*(d_nope*d_c + d_c*d_v)."""
+    return 2.0 * batch * cfg.chunk_tokens * cfg.n_heads * (cfg.d_nope * cfg.d_c + cfg.d_c * cfg.d_v)
 
 
 def peaks():
@@ -322,14 +331,12 @@ def _time(fn, reps, stream):
 def _fewstep_workload(V, synthetic, dev, stream, clocks, batch=1, n_chunks=14, n_denoise=4):
     """One Wan layer streaming n_chunks chunks, each denoised over n_denoise steps: the first step
     appends the chunk, the others rewrite it in place; every step attends with its own queries
-    (latent: compress -> absorb -> attention -> value-up; dense: project -> rope -> MHA)."""
+    (latent: compress -> fused absorb / attention / value-up; dense: project -> rope -> MHA)."""
     cfg, B = WAN, batch
     sets = [tuple(t.to(dev) for t in synthetic.draw_chunk(cfg, B, synthetic.rollout_seed(11, 0, k)))
             for k in range(n_denoise)]
     wd, wuk, wuv = (t.to(dev) for t in synthetic.draw_weights(cfg, 12))
     w_kv = synthetic.draw_dense_weights(cfg, 13).to(dev)
-    q_abs = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_qk), dtype=torch.bfloat16, device=dev)
-    o_lat = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_c), dtype=torch.bfloat16, device=dev)
     o = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
     dq = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_h), dtype=torch.bfloat16, device=dev)
     res = {}
@@ -348,9 +355,7 @@ def _fewstep_workload(V, synthetic, dev, stream, clocks, batch=1, n_chunks=14, n
                         V.compress_append(cfg, x, wd, cache)
                     else:
                         V.compress_rewrite(cfg, x, wd, cache)
-                    V.absorb_q(cfg, qn, qr, wuk, f0, out=q_abs)
-                    V.latent_attention(cfg, q_abs, cache, f0, out=o_lat)
-                    V.value_up(cfg, o_lat, wuv, out=o)
+                    V.latent_attention_fused(cfg, qn, qr, wuk, wuv, cache, f0, out=o)
                 else:
                     if s == 0:
                         f0 = cache.frames_written
@@ -383,8 +388,10 @@ def _capacity_workload(V, synthetic, dev, clocks, budget=60 * 10**9, n_layers=30
     for name, cfg, dense in (("latent_dc64", WAN.replace(d_c=64), False),
                              ("latent_dc128", WAN.replace(d_c=128), False),
                              ("latent_dc192", WAN, False), ("dense", WAN, True)):
-        plan = V.plan_capacity(cfg, n_layers, budget, dense=dense)
-        row = {"path": name, **plan}
+        # the latent step runs fused where the fused kernel supports the shape (d_c >= 128)
+        fused = (not dense) and cfg.d_c >= 128
+        plan = V.plan_capacity(cfg, n_layers, budget, dense=dense, fused=fused)
+        row = {"path": name + ("_fused" if fused else ""), **plan}
         if name in ("latent_dc192", "dense"):
             B = plan["max_batch"]
             torch.cuda.empty_cache()
@@ -412,7 +419,7 @@ def _capacity_workload(V, synthetic, dev, clocks, budget=60 * 10**9, n_layers=30
             del caches, out, x, qn, qr
             torch.cuda.empty_cache()
         rows.append(row)
-    by = {r["path"]: r["max_batch"] for r in rows}
+    by = {r["path"].replace("_fused", ""): r["max_batch"] for r in rows}
     return {"budget_bytes": budget, "n_layers": n_layers, "rows": rows,
             "batch_ratio_dc192_over_dense": by["latent_dc192"] / max(by["dense"], 1),
             "batch_ratio_dc64_over_dense": by["latent_dc64"] / max(by["dense"], 1)}
@@ -551,15 +558,23 @@ def main():
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    names = ["compress_append", "absorb_q", "latent_attention", "value_up"]
+    fused = args.path == "fused"
+    names = (["compress_append", "latent_attention_fused"] if fused else
+             ["compress_append", "absorb_q", "latent_attention", "value_up"])
+    n_ev = len(names) + 1
 
-    def step(i, ev=None):
-        x = xs[i % N_INPUT_SETS]
-        qn, qr = qs[i % N_INPUT_SETS]
+    def step(i, ev=None, x=None, qn=None, qr=None, use_fused=fused):
+        x = xs[i % N_INPUT_SETS] if x is None else x
+        if qn is None:
+            qn, qr = qs[i % N_INPUT_SETS]
         f0 = cache.frames_written
         if ev: ev[0].record(stream)
         V.compress_append(cfg, x, w, cache, f0)
         if ev: ev[1].record(stream)
+        if use_fused:
+            V.latent_attention_fused(cfg, qn, qr, w_uk, w_uv, cache, f0, out=bufs["o"])
+            if ev: ev[2].record(stream)
+            return
         V.absorb_q(cfg, qn, qr, w_uk, f0, out=bufs["q_abs"])
         if ev: ev[2].record(stream)
         V.latent_attention(cfg, bufs["q_abs"], cache, f0, out=bufs["o_latent"])
@@ -573,7 +588,7 @@ def main():
     torch.cuda.synchronize()
     assert V.device_status() == 0
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize()
@@ -589,27 +604,50 @@ def main():
     clk = clocks.stop()
     barrier(world)
     per_kernel = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)] for j, n in enumerate(names)}
-    step_ms = [evs[i][0].elapsed_time(evs[i][4]) for i in range(args.steps)]
+    step_ms = [evs[i][0].elapsed_time(evs[i][n_ev - 1]) for i in range(args.steps)]
     total_ms = max_over_ranks(sum(step_ms), world)
     assert V.device_status() == 0
 
     f_step = attention_flops(cfg, B)
     value = whole_job_rate(f_step, args.steps, world, total_ms) / 1e12
     q_tok_s = whole_job_rate(B * cfg.chunk_tokens, args.steps, world, total_ms)
-    k3_ms = statistics.mean(per_kernel["latent_attention"])
-    k3_tflops = f_step / (k3_ms * 1e-3) / 1e12
     kb = kernel_bytes(cfg, B)
-    kernels = {"latent_attention": {"ms": k3_ms, "tflops": k3_tflops}}
-    for n in ("compress_append", "absorb_q", "value_up"):
+    k3 = "latent_attention_fused" if fused else "latent_attention"
+    k3_ms = statistics.mean(per_kernel[k3])
+    # algorithmic flops of the dominant launch: the attention, plus the two projections when fused
+    k3_flops = f_step + (projection_flops(cfg, B) if fused else 0.0)
+    k3_tflops = k3_flops / (k3_ms * 1e-3) / 1e12
+    kernels = {k3: {"ms": k3_ms, "tflops": k3_tflops, "attention_tflops": f_step / (k3_ms * 1e-3) / 1e12}}
+    for n in names:
+        if n == k3:
+            continue
         ms = statistics.mean(per_kernel[n])
         kernels[n] = {"ms": ms, "gbs": kb[n] / (ms * 1e-3) / 1e9, "frac_hbm": kb[n] / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]}
     k3_src = source_hash(["tc_attention.cu", "tc_kernels.cuh", "ptx_sm100.cuh"])
-    roofline = {"bound": "tensor", "kernel": "latent_attention", "achieved": k3_tflops,
+    roofline = {"bound": "tensor", "kernel": k3, "achieved": k3_tflops,
                 "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": k3_tflops / pk["bf16_tflops"],
                 "peak_source": f"{pk_src} bf16 burst (MEASURED_PEAKS.json)" if pk_src == "measured" else "fallback 1.59 PFLOP/s",
                 "frac_of_sustained": k3_tflops / pk["bf16_tflops_sustained"],
-                "flops_per_launch": f_step,
-                "traffic": traffic_for("latent_attention_wan_b%d" % B, k3_src)}
+                "flops_per_launch": k3_flops,
+                "traffic": traffic_for("%s_wan_b%d" % (k3, B), k3_src)}
+
+    # ---- both paths on the same cache and inputs, interleaved step by step so that both see the same
+    # clock and power state (not part of `value`) ----
+    ab_steps = max(10, args.steps // 8)
+    ab = {True: [], False: []}
+    for i in range(2 * ab_steps):
+        use = (i % 4) in (0, 3)                   # fused, three, three, fused, ...
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.zero_()
+        a.record(stream)
+        step(args.warmup + args.steps + i, use_fused=use)
+        b.record(stream)
+        ab[use].append((a, b))
+    torch.cuda.synchronize()
+    path_ab = {"fused_step_ms": statistics.median(a.elapsed_time(b) for a, b in ab[True]),
+               "three_call_step_ms": statistics.median(a.elapsed_time(b) for a, b in ab[False]),
+               "steps_each": ab_steps}
+    path_ab["fused_over_three"] = path_ab["fused_step_ms"] / path_ab["three_call_step_ms"]
 
     # ---- end to end through the public API with host buffers (pinned) ----
     hx = [x.cpu().pin_memory() for x in xs]
@@ -623,11 +661,7 @@ def main():
         dx.copy_(hx[i % N_INPUT_SETS], non_blocking=True)
         dqn.copy_(hq[i % N_INPUT_SETS][0], non_blocking=True)
         dqr.copy_(hq[i % N_INPUT_SETS][1], non_blocking=True)
-        f0 = cache.frames_written
-        V.compress_append(cfg, dx, w, cache, f0)
-        V.absorb_q(cfg, dqn, dqr, w_uk, f0, out=bufs["q_abs"])
-        V.latent_attention(cfg, bufs["q_abs"], cache, f0, out=bufs["o_latent"])
-        V.value_up(cfg, bufs["o_latent"], w_uv, out=bufs["o"])
+        step(i, x=dx, qn=dqn, qr=dqr)
         ho.copy_(bufs["o"], non_blocking=True)
 
     for i in range(3):
@@ -683,6 +717,7 @@ def main():
         comparison = {"dense_step_ms": d_step_ms, "dense_mha_ms": d_mha_ms,
                       "dense_mha_tflops": dense_attention_flops(cfg, B) / (d_mha_ms * 1e-3) / 1e12,
                       "latent_step_ms": statistics.mean(step_ms), "latent_attention_ms": k3_ms,
+                      "latent_attention_includes_projections": fused,
                       "step_speedup_vs_dense": d_step_ms / statistics.mean(step_ms),
                       "attention_speedup_vs_dense": d_mha_ms / k3_ms,
                       "cache_bytes_latent": V.latent_cache_bytes(cfg, B),
@@ -702,11 +737,14 @@ def main():
                            "query_tokens": cfg.chunk_tokens, "cached_tokens": cfg.window_tokens,
                            "heads": cfg.n_heads, "d_c": cfg.d_c, "d_rope": cfg.d_rope, "d_v": cfg.d_v,
                            "dim": cfg.dim, "parallelism": f"dp{world} (independent sequences)",
-                           "l2": "flushed between steps (512 MB write)"},
+                           "l2": "flushed between steps (512 MB write)",
+                           "path": ("compress + fused absorb/attention/value-up" if fused
+                                    else "compress + absorb + attention + value-up")},
                 "query_tokens_per_s": q_tok_s,
                 "pct_of_bf16_peak": 100.0 * value / world / pk["bf16_tflops"],
                 "roofline": roofline, "kernels": kernels, "e2e": e2e, "gpu_launches": launches,
-                "clocks": clk, "wall_s_timed": wall, "cpu_baseline": cpu, "comparison": comparison}
+                "clocks": clk, "wall_s_timed": wall, "cpu_baseline": cpu, "path_ab": path_ab,
+                "comparison": comparison}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

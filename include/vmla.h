@@ -205,22 +205,28 @@ VMLA_API int64_t vmla_dense_cache_bytes(const vmla_config* cfg, int32_t batch);
 
 /* Largest batch that fits a fixed memory budget (the technical summary's Results, "Scalability": at a
  * fixed B200 memory budget the latent cache admits a much larger batch than dense MHA).  For a model of
- * n_layers attention layers of this shape (dense = 0: latent path, 1: dense MHA path):
+ * n_layers attention layers of this shape, stepped along `path` (a vmla_path):
  *   per sequence  cache   n_layers * W*T_f * (d_c + d_rope)  or  n_layers * W*T_f * n_heads*(d_h + d_v)
  *                 buffers the tensors of one layer step, reused across layers (x [F*T_f, dim] and,
- *                         latent: q_nope, q_rope, q_abs, out_latent, out; dense: q, out)
+ *                         latent: q_nope, q_rope, q_abs, out_latent, out; latent fused: q_nope,
+ *                         q_rope, out; dense: q, out)
  *                 + extra_bytes_per_seq (activations outside this library)
  *   fixed         this library's weights for n_layers layers (latent: w_dkv_kr, w_uk, w_uv; dense:
  *                 w_kv) + fixed_bytes (the rest of the model)
  * all in the storage type of cfg->dtype.  out->max_batch = floor((budget - fixed) / per sequence),
  * 0 when the fixed bytes alone exceed the budget.  Host-only; launches nothing. */
+typedef enum {
+  VMLA_PATH_LATENT = 0,        /* compress, absorb, latent attention, value up-projection */
+  VMLA_PATH_DENSE = 1,         /* dense projection, rope, dense MHA */
+  VMLA_PATH_LATENT_FUSED = 2   /* compress, vmla_latent_attention_fused */
+} vmla_path;
 typedef struct {
   int64_t max_batch;
   int64_t cache_bytes_per_seq;   /* all layers' cache of one sequence */
   int64_t buffer_bytes_per_seq;  /* one layer step's tensors for one sequence */
   int64_t weight_bytes;          /* this library's weights, all layers */
 } vmla_capacity;
-VMLA_API vmla_status vmla_plan_capacity(const vmla_config* cfg, int32_t n_layers, int32_t dense,
+VMLA_API vmla_status vmla_plan_capacity(const vmla_config* cfg, int32_t n_layers, int32_t path,
                                         int64_t budget_bytes, int64_t fixed_bytes,
                                         int64_t extra_bytes_per_seq, vmla_capacity* out);
 

@@ -171,13 +171,16 @@ int64_t vmla_dense_cache_bytes(const vmla_config* cfg, int32_t batch) {
          (cfg->d_nope + cfg->d_rope + cfg->d_v) * elt;
 }
 
-vmla_status vmla_plan_capacity(const vmla_config* cfg, int32_t n_layers, int32_t dense,
+vmla_status vmla_plan_capacity(const vmla_config* cfg, int32_t n_layers, int32_t path,
                                int64_t budget_bytes, int64_t fixed_bytes, int64_t extra_bytes_per_seq,
                                vmla_capacity* out) {
   vmla_status s = check_config(cfg);
   if (s != VMLA_OK) return s;
   if (!out) return fail(VMLA_ERR_INVALID_ARG, "out is NULL");
   if (n_layers <= 0) return fail(VMLA_ERR_INVALID_ARG, "n_layers must be >= 1");
+  if (path < VMLA_PATH_LATENT || path > VMLA_PATH_LATENT_FUSED)
+    return fail(VMLA_ERR_INVALID_ARG, "path must be VMLA_PATH_LATENT, VMLA_PATH_DENSE or VMLA_PATH_LATENT_FUSED");
+  const bool dense = path == VMLA_PATH_DENSE;
   if (budget_bytes < 0 || fixed_bytes < 0 || extra_bytes_per_seq < 0)
     return fail(VMLA_ERR_INVALID_ARG, "budget, fixed and extra bytes must be >= 0");
   const int64_t elt = cfg->dtype == VMLA_BF16 ? 2 : 4;
@@ -192,8 +195,8 @@ vmla_status vmla_plan_capacity(const vmla_config* cfg, int32_t n_layers, int32_t
   } else {
     const int64_t dc = cfg->d_c, dr = cfg->d_rope;
     cache_tok = dc + dr;
-    buffers = nq * D + nq * H * cfg->d_nope + nq * H * dr + nq * H * (dc + dr)  // x, q_nope, q_rope, q_abs
-              + nq * H * dc + nq * H * dv;                                      // out_latent, out
+    buffers = nq * D + nq * H * cfg->d_nope + nq * H * dr + nq * H * dv;      // x, q_nope, q_rope, out
+    if (path == VMLA_PATH_LATENT) buffers += nq * H * (dc + dr) + nq * H * dc;  // q_abs, out_latent
     weights = (dc + dr) * D + H * cfg->d_nope * dc + H * dv * dc;               // w_dkv_kr, w_uk, w_uv
   }
   out->cache_bytes_per_seq = (int64_t)n_layers * nk * cache_tok * elt;

@@ -374,25 +374,33 @@ def dense_cache_bytes(cfg: VmlaConfig, batch: int) -> int:
 
 
 def plan_capacity(cfg: VmlaConfig, n_layers: int, budget_bytes: int, *, dense: bool = False,
-                  fixed_bytes: int = 0, extra_bytes_per_seq: int = 0) -> dict:
+                  fused: bool = False, fixed_bytes: int = 0, extra_bytes_per_seq: int = 0) -> dict:
     """Largest batch of sequences whose n_layers caches, one layer step's tensors and the given extra
-    bytes fit ``budget_bytes`` (host-only; see vmla_plan_capacity)."""
+    bytes fit ``budget_bytes`` (host-only; see vmla_plan_capacity).  dense: the dense MHA path;
+    fused: the latent path through vmla_latent_attention_fused."""
     cc = c_config(cfg)
     out = CCapacity()
-    check(LIB.vmla_plan_capacity(ctypes.byref(cc), n_layers, 1 if dense else 0, int(budget_bytes),
+    path = 1 if dense else (2 if fused else 0)
+    check(LIB.vmla_plan_capacity(ctypes.byref(cc), n_layers, path, int(budget_bytes),
                                  int(fixed_bytes), int(extra_bytes_per_seq), ctypes.byref(out)))
     return {n: int(getattr(out, n)) for n, _ in CCapacity._fields_}
 
 
 def layer_step(cfg: VmlaConfig, x: torch.Tensor, q_nope: torch.Tensor, q_rope: torch.Tensor,
                w_dkv_kr: torch.Tensor, w_uk: torch.Tensor, w_uv: torch.Tensor, cache: LatentCache,
-               bufs: Optional[dict] = None) -> torch.Tensor:
+               bufs: Optional[dict] = None, fused: Optional[bool] = None) -> torch.Tensor:
     """One streaming step of one layer: append the chunk x, then attend with its queries and project
     the values up.  Returns o [B, F*T_f, H, d_v].  ``bufs`` (optional) holds reusable outputs under the
-    keys q_abs, o_latent, o."""
+    keys q_abs, o_latent, o.  ``fused`` selects the single-launch absorb + attention + value-up kernel
+    (default: for bf16 configs whose shapes it supports) or the three separate calls."""
     bufs = bufs if bufs is not None else {}
+    if fused is None:
+        fused = cfg.dtype == VMLA_BF16 and cfg.d_rope == 32 and cfg.d_c in (128, 192, 256) and \
+            cfg.d_nope % 16 == 0 and 16 <= cfg.d_nope <= 128 and cfg.d_v % 32 == 0 and 32 <= cfg.d_v <= 128
     f0 = cache.frames_written
     compress_append(cfg, x, w_dkv_kr, cache, f0)
+    if fused:
+        return latent_attention_fused(cfg, q_nope, q_rope, w_uk, w_uv, cache, f0, out=bufs.get("o"))
     q_abs = absorb_q(cfg, q_nope, q_rope, w_uk, f0, 1, out=bufs.get("q_abs"))
     o_lat = latent_attention(cfg, q_abs, cache, f0, 1, out=bufs.get("o_latent"))
     return value_up(cfg, o_lat, w_uv, out=bufs.get("o"))

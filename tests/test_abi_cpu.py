@@ -146,15 +146,16 @@ def test_rewrite_rejects_before_any_append():
 def test_plan_capacity_matches_oracle(cfg):
     from oracle import vmla_oracle as O
     elt = 2 if cfg.dtype != VMLA_F32 else 4
-    for dense in (False, True):
+    for dense, fused in ((False, False), (True, False), (False, True)):
         for n_layers, budget, fixed, extra in ((30, 180 * 10**9, 0, 0), (30, 180 * 10**9, 2_600_000_000, 300_000_000),
                                                (1, 10**6, 0, 0), (4, 5 * 10**8, 10**7, 12345), (30, 10**9, 2 * 10**9, 0)):
-            got = V.plan_capacity(cfg, n_layers, budget, dense=dense, fixed_bytes=fixed, extra_bytes_per_seq=extra)
+            got = V.plan_capacity(cfg, n_layers, budget, dense=dense, fused=fused, fixed_bytes=fixed,
+                                  extra_bytes_per_seq=extra)
             want = O.batch_capacity(budget, n_layers=n_layers, window_tokens=cfg.window_tokens, elt_bytes=elt,
                                     fixed_bytes=fixed, extra_bytes_per_seq=extra, dim=cfg.dim,
                                     n_heads=cfg.n_heads, d_nope=cfg.d_nope, d_rope=cfg.d_rope, d_c=cfg.d_c,
-                                    d_v=cfg.d_v, tokens_per_chunk=cfg.chunk_tokens, dense=dense)
-            assert got["max_batch"] == want, (dense, n_layers, budget, fixed, extra)
+                                    d_v=cfg.d_v, tokens_per_chunk=cfg.chunk_tokens, dense=dense, fused=fused)
+            assert got["max_batch"] == want, (dense, fused, n_layers, budget, fixed, extra)
     one = V.plan_capacity(cfg, 30, 10**12)
     assert one["cache_bytes_per_seq"] == 30 * V.latent_cache_bytes(cfg, 1)
     assert V.plan_capacity(cfg, 30, 10**12, dense=True)["cache_bytes_per_seq"] == 30 * V.dense_cache_bytes(cfg, 1)
@@ -163,7 +164,8 @@ def test_plan_capacity_matches_oracle(cfg):
 def test_plan_capacity_rejects_bad_arguments():
     cc = V.c_config(WAN)
     out = V.CCapacity()
-    for args in ((0, 0, 10, 0, 0), (30, 0, -1, 0, 0), (30, 0, 10, -5, 0), (30, 1, 10, 0, -1)):
+    for args in ((0, 0, 10, 0, 0), (30, 0, -1, 0, 0), (30, 0, 10, -5, 0), (30, 1, 10, 0, -1), (30, 3, 10, 0, 0),
+                 (30, -1, 10, 0, 0)):
         st, _ = _status(V.LIB.vmla_plan_capacity, ctypes.byref(cc), *args, ctypes.byref(out))
         assert st == V.VMLA_ERR_INVALID_ARG
     st, _ = _status(V.LIB.vmla_plan_capacity, ctypes.byref(cc), 30, 0, 10, 0, 0, None)

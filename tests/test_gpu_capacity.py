@@ -19,7 +19,7 @@ def V():
     return vmla
 
 
-def _held_bytes(V, cfg, batch, n_layers, dense):
+def _held_bytes(V, cfg, batch, n_layers, dense, fused=False):
     """Device bytes held by n_layers caches and one layer step of ``batch`` sequences."""
     torch.cuda.synchronize()
     base = torch.cuda.memory_allocated()
@@ -37,10 +37,14 @@ def _held_bytes(V, cfg, batch, n_layers, dense):
         w, w_uk, w_uv = (t.to(DEV) for t in synthetic.draw_weights(cfg, 6))
         weights = sum(t.numel() * t.element_size() for t in (w, w_uk, w_uv))
         V.compress_append(cfg, x, w, caches[0])
-        q_abs = V.absorb_q(cfg, qn, qr, w_uk, 0)
-        o_lat = V.latent_attention(cfg, q_abs, caches[0], 0)
-        out = V.value_up(cfg, o_lat, w_uv)
-        held = [x, qn, qr, q_abs, o_lat, out, caches]
+        if fused:
+            out = V.latent_attention_fused(cfg, qn, qr, w_uk, w_uv, caches[0], 0)
+            held = [x, qn, qr, out, caches]
+        else:
+            q_abs = V.absorb_q(cfg, qn, qr, w_uk, 0)
+            o_lat = V.latent_attention(cfg, q_abs, caches[0], 0)
+            out = V.value_up(cfg, o_lat, w_uv)
+            held = [x, qn, qr, q_abs, o_lat, out, caches]
         base += weights
     torch.cuda.synchronize()
     if dense:
@@ -48,15 +52,16 @@ def _held_bytes(V, cfg, batch, n_layers, dense):
     return torch.cuda.memory_allocated() - base, held
 
 
-@pytest.mark.parametrize("dense", [False, True], ids=["latent", "dense"])
-def test_planner_bytes_per_sequence_match_device_allocation(V, dense):
+@pytest.mark.parametrize("dense,fused", [(False, False), (True, False), (False, True)],
+                         ids=["latent", "dense", "latent_fused"])
+def test_planner_bytes_per_sequence_match_device_allocation(V, dense, fused):
     cfg, n_layers = MID, 3
-    a, held_a = _held_bytes(V, cfg, 2, n_layers, dense)
+    a, held_a = _held_bytes(V, cfg, 2, n_layers, dense, fused)
     del held_a
     torch.cuda.empty_cache()
-    b, held_b = _held_bytes(V, cfg, 3, n_layers, dense)
+    b, held_b = _held_bytes(V, cfg, 3, n_layers, dense, fused)
     del held_b
-    plan = V.plan_capacity(cfg, n_layers, 10**12, dense=dense)
+    plan = V.plan_capacity(cfg, n_layers, 10**12, dense=dense, fused=fused)
     per_seq = plan["cache_bytes_per_seq"] + plan["buffer_bytes_per_seq"]
     # the caching allocator rounds each block up to 512 bytes
     assert abs((b - a) - per_seq) <= 512 * 16, (b - a, per_seq)
