@@ -230,6 +230,31 @@ VMLA_API vmla_status vmla_plan_capacity(const vmla_config* cfg, int32_t n_layers
                                         int64_t budget_bytes, int64_t fixed_bytes,
                                         int64_t extra_bytes_per_seq, vmla_capacity* out);
 
+/* ---- Streaming executor: layer steps whose inputs and outputs are in host memory ----
+ * Each submitted step copies x [batch, F*T_f, dim], q_nope [batch, F*T_f, n_heads, d_nope] and
+ * q_rope [batch, F*T_f, n_heads, d_rope] from the host, runs vmla_compress_append and
+ * vmla_latent_attention_fused on `cache` with the given weights (device pointers, layouts as in those
+ * calls), and copies o [batch, F*T_f, n_heads, d_v] back to out_host.  Two staging slots in the
+ * caller's device workspace let the copies of the neighbouring steps overlap this step's kernels: the
+ * host -> device copies run on one internal stream, the device -> host copies on another, the kernels
+ * on the stream given at creation; events order the three.  Steps may use different caches and
+ * weights (one executor can serve every layer).
+ * Ownership: the workspace (>= vmla_executor_workspace_bytes(), 256-byte aligned) and every buffer
+ * stay the caller's; the executor owns only its two streams and six events.  Host buffers should be
+ * page-locked (pageable memory makes the copies synchronous); an input buffer may be reused, and
+ * out_host read, only after vmla_executor_wait().  cache->frames_written advances at submit.
+ * bf16 only (VMLA_ERR_UNSUPPORTED otherwise); errors of the inner calls are returned as they are. */
+typedef struct vmla_executor vmla_executor;
+VMLA_API int64_t vmla_executor_workspace_bytes(const vmla_config* cfg, int32_t batch);   /* -1 on bad args */
+VMLA_API vmla_status vmla_executor_create(const vmla_config* cfg, int32_t batch, void* workspace,
+                                          int64_t workspace_bytes, void* stream, vmla_executor** out);
+VMLA_API vmla_status vmla_executor_submit(vmla_executor* ex, vmla_cache* cache, const void* w_dkv_kr,
+                                          const void* w_uk, const void* w_uv, const void* x_host,
+                                          const void* q_nope_host, const void* q_rope_host, void* out_host);
+/* Blocks until every submitted step's output is in host memory; then as vmla_device_status(). */
+VMLA_API vmla_status vmla_executor_wait(vmla_executor* ex);
+VMLA_API vmla_status vmla_executor_destroy(vmla_executor* ex);   /* waits for pending copies first */
+
 /* Set the bound of every device-side wait of later launches to `ms` milliseconds (default 1000) and
  * return the previous bound; ms <= 0 only returns the current bound.  A wait that runs out makes the
  * kernel stop, record a nonzero code for vmla_device_status() and return. */

@@ -481,7 +481,13 @@ cudaError_t tc_compress_append(const vmla_config& cfg, int batch, const void* x,
   const int64_t ntok = (int64_t)cfg.chunk_frames * cfg.grid_h * cfg.grid_w;
   const int64_t M = batch * ntok;
   const int N = cfg.d_c + cfg.d_rope, K = cfg.dim;
-  const int bn = pick_bn(N);
+  // one 224-wide column tile per 128 rows leaves most SMs idle at small batch: narrow the column tile
+  // until the tiles cover the SMs (the x tile is then re-read from L2 by each column tile; the RoPE
+  // columns d_c .. d_c+31 stay inside one 32-column chunk of one tile because d_c % 32 == 0)
+  int bn = pick_bn(N);
+  const int64_t m_tiles = (M + kBM - 1) / kBM;
+  for (int cand : {128, 64})
+    if (m_tiles * ((N + bn - 1) / bn) < num_sms() && cand < bn) bn = cand;
   CUtensorMap ma, mb;
   cudaError_t e;
   // A = x [M, D]; B = [W^KV_down ; W^KR] [N, D], both K-major

@@ -121,6 +121,8 @@ cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+vmla_status report(vmla_status s, const char* what) { return fail(s, "%s", what); }
+
 int* device_status_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;

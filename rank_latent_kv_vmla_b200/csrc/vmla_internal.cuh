@@ -85,6 +85,7 @@ __device__ __forceinline__ void rope_rotate_f32(const RopeTable& rt, int p, int6
 // Device status word (bounded waits that ran out record a nonzero code here).
 int* device_status_ptr();   // address of this device's status word (host side), nullptr on error
 void count_launches(int n);
+vmla_status report(vmla_status s, const char* what);   // sets the thread's error detail, returns s
 
 // ------------------------------------------------------------------------------------------------
 // CUDA-core kernels (fp32 path)

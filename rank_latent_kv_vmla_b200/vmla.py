@@ -25,7 +25,8 @@ EXPORTED = ("vmla_compress_append", "vmla_absorb_q", "vmla_latent_attention", "v
             "vmla_latent_cache_bytes", "vmla_dense_cache_bytes", "vmla_launch_count",
             "vmla_status_string", "vmla_last_error_detail", "vmla_abi_version",
             "vmla_compress_rewrite", "vmla_dense_rewrite", "vmla_plan_capacity",
-            "vmla_latent_attention_fused")
+            "vmla_latent_attention_fused", "vmla_executor_workspace_bytes", "vmla_executor_create",
+            "vmla_executor_submit", "vmla_executor_wait", "vmla_executor_destroy")
 
 
 class VmlaError(RuntimeError):
@@ -79,6 +80,10 @@ def _load():
         "vmla_dense_rewrite": [cfgp, VP, VP, P(CDenseCache), VP],
         "vmla_plan_capacity": [cfgp, I32, I32, I64, I64, I64, P(CCapacity)],
         "vmla_latent_attention_fused": [cfgp, VP, VP, VP, VP, P(CCache), I64, I32, VP, VP, VP],
+        "vmla_executor_create": [cfgp, I32, VP, I64, VP, P(VP)],
+        "vmla_executor_submit": [VP, P(CCache), VP, VP, VP, VP, VP, VP, VP],
+        "vmla_executor_wait": [VP],
+        "vmla_executor_destroy": [VP],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -87,6 +92,8 @@ def _load():
     for name in ("vmla_latent_cache_bytes", "vmla_dense_cache_bytes"):
         getattr(lib, name).argtypes = [cfgp, I32]
         getattr(lib, name).restype = I64
+    lib.vmla_executor_workspace_bytes.argtypes = [cfgp, I32]
+    lib.vmla_executor_workspace_bytes.restype = I64
     lib.vmla_launch_count.argtypes = []
     lib.vmla_launch_count.restype = I64
     lib.vmla_status_string.argtypes = [ctypes.c_int]
@@ -386,6 +393,71 @@ def plan_capacity(cfg: VmlaConfig, n_layers: int, budget_bytes: int, *, dense: b
     return {n: int(getattr(out, n)) for n, _ in CCapacity._fields_}
 
 
+class Executor:
+    """Streaming executor of the C library: layer steps with inputs and outputs in (pinned) host memory,
+    the copies of neighbouring steps overlapping each step's kernels.  The device workspace is allocated
+    here with PyTorch; kernels run on the current stream at creation."""
+
+    def __init__(self, cfg: VmlaConfig, batch: int, device="cuda"):
+        self.cfg, self.batch = cfg, batch
+        cc = c_config(cfg)
+        nbytes = int(LIB.vmla_executor_workspace_bytes(ctypes.byref(cc), batch))
+        if nbytes < 0:
+            raise VmlaError(VMLA_ERR_INVALID_ARG, "bad executor arguments")
+        self.workspace = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        base = self.workspace.data_ptr()
+        aligned = (base + 255) // 256 * 256
+        self._stream = torch.cuda.current_stream(self.workspace.device)
+        handle = ctypes.c_void_p()
+        check(LIB.vmla_executor_create(ctypes.byref(cc), batch, aligned, nbytes, self._stream.cuda_stream,
+                                       ctypes.byref(handle)))
+        self._h = handle
+        self._keep = []
+
+    def submit(self, cache: LatentCache, w_dkv_kr, w_uk, w_uv, x_host, q_nope_host, q_rope_host, out_host):
+        cfg = self.cfg
+        for t, name in ((x_host, "x_host"), (q_nope_host, "q_nope_host"), (q_rope_host, "q_rope_host"),
+                        (out_host, "out_host")):
+            if t.is_cuda or not t.is_contiguous() or t.dtype != _dtype(cfg):
+                raise ValueError(f"{name} must be a contiguous host tensor of {_dtype(cfg)}")
+        B, n, H = self.batch, cfg.chunk_tokens, cfg.n_heads
+        shapes = ((x_host, (B, n, cfg.dim)), (q_nope_host, (B, n, H, cfg.d_nope)),
+                  (q_rope_host, (B, n, H, cfg.d_rope)), (out_host, (B, n, H, cfg.d_v)))
+        for t, shp in shapes:
+            if tuple(t.shape) != shp:
+                raise ValueError(f"host tensor has shape {tuple(t.shape)}, expected {shp}")
+        check(LIB.vmla_executor_submit(self._h, ctypes.byref(cache.struct),
+                                       _arg(w_dkv_kr, cfg, (cfg.d_c + cfg.d_rope, cfg.dim), "w_dkv_kr"),
+                                       _arg(w_uk, cfg, (H, cfg.d_nope, cfg.d_c), "w_uk"),
+                                       _arg(w_uv, cfg, (H, cfg.d_v, cfg.d_c), "w_uv"),
+                                       x_host.data_ptr(), q_nope_host.data_ptr(), q_rope_host.data_ptr(),
+                                       out_host.data_ptr()))
+        self._keep.append((x_host, q_nope_host, q_rope_host, out_host))
+
+    def wait(self) -> None:
+        st = LIB.vmla_executor_wait(self._h)
+        self._keep.clear()
+        check(st)
+
+    def close(self) -> None:
+        if self._h is not None:
+            LIB.vmla_executor_destroy(self._h)
+            self._h = None
+            self._keep.clear()
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
 def layer_step(cfg: VmlaConfig, x: torch.Tensor, q_nope: torch.Tensor, q_rope: torch.Tensor,
                w_dkv_kr: torch.Tensor, w_uk: torch.Tensor, w_uv: torch.Tensor, cache: LatentCache,
                bufs: Optional[dict] = None, fused: Optional[bool] = None) -> torch.Tensor:
@@ -409,5 +481,5 @@ def layer_step(cfg: VmlaConfig, x: torch.Tensor, q_nope: torch.Tensor, q_rope: t
 __all__ = ["LIB", "VmlaError", "LatentCache", "DenseCache", "compress_append", "absorb_q",
            "latent_attention", "value_up", "rope_q", "dense_append", "dense_mha", "device_status",
            "launch_count", "latent_cache_bytes", "dense_cache_bytes", "layer_step", "c_config",
-           "compress_rewrite", "dense_rewrite", "plan_capacity", "CCapacity", "latent_attention_fused",
+           "compress_rewrite", "dense_rewrite", "plan_capacity", "CCapacity", "latent_attention_fused", "Executor",
            "CConfig", "CCache", "CDenseCache", "EXPORTED", "VMLA_F32", "VMLA_BF16"]

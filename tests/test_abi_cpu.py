@@ -189,3 +189,24 @@ def test_fused_attention_rejects_unsupported_shapes():
     st, _ = _status(V.LIB.vmla_latent_attention_fused, ctypes.byref(cc), FAKE + 8, FAKE, FAKE, FAKE,
                     ctypes.byref(_cache(frames_written=3)), 0, 1, FAKE, None, None)
     assert st == V.VMLA_ERR_MISALIGNED
+
+
+def test_executor_workspace_and_rejections():
+    """Workspace arithmetic (two slots of x, q_nope, q_rope, out, each 256-byte rounded) and the
+    argument checks that run before any CUDA call."""
+    cc = V.c_config(WAN)
+    n = WAN.chunk_tokens
+    per = [n * WAN.dim * 2, n * 12 * 96 * 2, n * 12 * 32 * 2, n * 12 * 128 * 2]
+    slot = sum((b + 255) // 256 * 256 for b in per)
+    assert V.LIB.vmla_executor_workspace_bytes(ctypes.byref(cc), 1) == 2 * slot
+    assert V.LIB.vmla_executor_workspace_bytes(ctypes.byref(cc), 0) == -1
+    h = ctypes.c_void_p()
+    st, _ = _status(V.LIB.vmla_executor_create, ctypes.byref(V.c_config(TINY)), 1, 0x100000, 1 << 30, None,
+                    ctypes.byref(h))
+    assert st == V.VMLA_ERR_UNSUPPORTED and not h.value
+    st, _ = _status(V.LIB.vmla_executor_create, ctypes.byref(cc), 1, 0x100000 + 16, 1 << 30, None, ctypes.byref(h))
+    assert st == V.VMLA_ERR_MISALIGNED
+    st, _ = _status(V.LIB.vmla_executor_create, ctypes.byref(cc), 1, 0x100000, 1024, None, ctypes.byref(h))
+    assert st == V.VMLA_ERR_INVALID_ARG
+    assert V.LIB.vmla_executor_wait(None) == V.VMLA_ERR_INVALID_ARG
+    assert V.LIB.vmla_executor_destroy(None) == V.VMLA_OK
