@@ -47,6 +47,10 @@ def parse():
     ap.add_argument("--batch", type=int, default=1, help="sequences per GPU")
     ap.add_argument("--impl", default="vmla", choices=["vmla", "reference"])
     ap.add_argument("--no-dense", action="store_true", help="skip the dense MHA comparison arm")
+    ap.add_argument("--parallel", default="batch", choices=["batch", "query"],
+                    help="batch: each rank runs its own sequences (weak scaling, no collective); query: one "
+                         "batch whose chunk query rows are sharded over the ranks, each holding a replica of "
+                         "the latent cache that every rank's compress kernel writes (strong scaling)")
     ap.add_argument("--path", default="fused", choices=["fused", "three"],
                     help="fused: compress + one fused attention launch per step; three: compress + "
                          "absorb + attention + value-up launches (the other path is timed beside it)")
@@ -525,12 +529,90 @@ def run_workload(args):
     print(json.dumps(out), flush=True)
 
 
+def run_query_sharded(args):
+    """--parallel query: one batch of B sequences; every rank compresses and attends its token range of
+    each chunk (rank_latent_kv_vmla_b200.sharding).  value = the whole chunk's latent-attention flops per
+    second of the slowest rank (strong scaling: the work does not grow with the ranks)."""
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    rank, world, local = dist_setup("nccl")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from rank_latent_kv_vmla_b200 import vmla as V
+    from rank_latent_kv_vmla_b200.sharding import ShardedLayer, TorchComm
+    import synthetic
+    cfg, B = WAN, args.batch
+    pk, pk_src = peaks()
+    seed = rank_seed(0)                                   # every rank draws the same sequence
+    prefill = cfg.window_frames // cfg.chunk_frames - 1
+    inp = synthetic.draw_layer(cfg, batch=B, seed=seed, n_chunks=prefill + N_INPUT_SETS)
+    extra_q = [synthetic.draw_queries(cfg, B, seed + 7 + i) for i in range(N_INPUT_SETS)]
+    w, w_uk, w_uv = inp.w_dkv_kr.to(dev), inp.w_uk.to(dev), inp.w_uv.to(dev)
+    comm = TorchComm(device=dev)
+    layer = ShardedLayer(cfg, B, comm, device=dev)
+    b0, cnt = layer.begin, layer.count
+    rows = lambda t: t[:, b0:b0 + cnt].contiguous().to(dev)
+    xs = [rows(x) for x in inp.x_chunks]
+    qs = [(rows(qn), rows(qr)) for qn, qr in extra_q]
+    out = torch.empty((B, max(cnt, 1), cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)[:, :cnt]
+    for k in range(prefill):
+        layer.step(xs[k], qs[0][0], qs[0][1], w, w_uk, w_uv, out=out if cnt else None)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, ev=None):
+        j = i % N_INPUT_SETS
+        if ev: ev[0].record(stream)
+        layer.step(xs[prefill + j], qs[j][0], qs[j][1], w, w_uk, w_uv, out=out if cnt else None)
+        if ev: ev[1].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+        flush.zero_()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    launches0 = V.launch_count()
+    for i in range(args.steps):
+        step(args.warmup + i, evs[i])
+        flush.zero_()
+    torch.cuda.synchronize()
+    launches = V.launch_count() - launches0
+    clk = clocks.stop()
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs), world)
+    assert V.device_status() == 0
+    layer.close()
+    f_step = attention_flops(cfg, B)
+    value = f_step * args.steps / (total_ms * 1e-3) / 1e12
+    if rank == 0:
+        line = {"metric": "latent-attention TFLOP/s (Wan-1.3B layer step, B200 BF16 TC peak fraction)",
+                "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "strong",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "wan1.3b_layer_stream_step", "batch": B, "query_tokens": cfg.chunk_tokens,
+                           "cached_tokens": cfg.window_tokens, "heads": cfg.n_heads, "d_c": cfg.d_c,
+                           "parallelism": f"query rows sharded over {world} GPUs, latent cache replicated",
+                           "shards": layer.shards, "l2": "flushed between steps (512 MB write)"},
+                "query_tokens_per_s": B * cfg.chunk_tokens * args.steps / (total_ms * 1e-3),
+                "pct_of_bf16_peak": 100.0 * value / world / pk["bf16_tflops"],
+                "gpu_launches": launches, "clocks": clk, "e2e": None, "cpu_baseline": None}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.workload != "layer":
         return run_workload(args)
+    if args.parallel == "query":
+        return run_query_sharded(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     rank, world, local = dist_setup("nccl")

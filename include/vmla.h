@@ -104,6 +104,33 @@ typedef struct {
 VMLA_API vmla_status vmla_compress_append(const vmla_config* cfg, const void* x, const void* w_dkv_kr,
                                  int64_t first_frame, vmla_cache* cache, void* stream);
 
+/* One sequence on several GPUs (query-row sharding, replicated cache; the technical summary's Problem
+ * definition: a fixed-size sliding window per sequence): every GPU holds a full replica of the latent
+ * cache and compresses only a token range of each chunk.  This call compresses tokens token_begin ..
+ * token_begin+n_tokens-1 of the chunk of frames first_frame .. first_frame+F-1 and stores each token's
+ * c and k^R rows into the rings of all n_replicas caches (1..8).  Replica planes on other GPUs are
+ * reached through peer mappings (vmla_ipc_import) with plain stores, so the compute and the exchange of
+ * the new latents are one kernel; the caller orders that kernel before any reader on another GPU (for
+ * example with a collective on the same stream) and then advances frames_written of every replica by
+ * F itself: this call does not.
+ *   x_rows [batch, n_tokens, dim]; w_dkv_kr as in vmla_compress_append; replicas[r].frames_written
+ *   must all equal first_frame.  bf16 only. */
+VMLA_API vmla_status vmla_compress_append_rows(const vmla_config* cfg, const void* x_rows, const void* w_dkv_kr,
+                                               int64_t first_frame, int64_t token_begin, int64_t n_tokens,
+                                               const vmla_cache* replicas, int32_t n_replicas, void* stream);
+
+/* Peer mappings of device buffers across processes (CUDA IPC).  vmla_ipc_export describes the buffer
+ * holding dev_ptr (allocation handle + offset of dev_ptr in it); vmla_ipc_import maps it into this
+ * process (another GPU's memory, reached over NVLink) and returns the matching pointer;
+ * vmla_ipc_release unmaps it.  The exporter keeps its buffer alive until every importer released it. */
+typedef struct {
+  unsigned char bytes[64];
+  int64_t offset;
+} vmla_ipc_handle;
+VMLA_API vmla_status vmla_ipc_export(const void* dev_ptr, vmla_ipc_handle* out);
+VMLA_API vmla_status vmla_ipc_import(const vmla_ipc_handle* h, void** dev_ptr);
+VMLA_API vmla_status vmla_ipc_release(void* dev_ptr);
+
 /* Few-step generation: recompute the newest chunk's cache rows in place.  Streaming video diffusion
  * denoises each chunk over several steps (the technical summary's Problem definition names
  * Self-Forcing-style training); at every step the chunk's own keys come from that step's features,
@@ -152,6 +179,16 @@ VMLA_API vmla_status vmla_latent_attention_fused(const vmla_config* cfg, const v
                                                  const void* w_uk, const void* w_uv, const vmla_cache* cache,
                                                  int64_t first_frame, int32_t n_query_chunks, void* out,
                                                  float* lse, void* stream);
+
+/* vmla_latent_attention_fused for the query tokens token_begin .. token_begin+n_tokens-1 of the call
+ * only (a shard of the rows): q_nope [batch, n_tokens, n_heads, d_nope], q_rope [batch, n_tokens,
+ * n_heads, d_rope] -> out [batch, n_tokens, n_heads, d_v], lse [batch, n_tokens, n_heads].  Positions and
+ * the window rule are those of the tokens' place in the call. */
+VMLA_API vmla_status vmla_latent_attention_fused_rows(const vmla_config* cfg, const void* q_nope,
+                                                      const void* q_rope, const void* w_uk, const void* w_uv,
+                                                      const vmla_cache* cache, int64_t first_frame,
+                                                      int32_t n_query_chunks, int64_t token_begin,
+                                                      int64_t n_tokens, void* out, float* lse, void* stream);
 
 /* Value up-projection applied once to the attention-weighted latent (VideoMLA, Method item 2):
  *   out[b, n, h, :] = W^V_up,h out_latent[b, n, h, :]

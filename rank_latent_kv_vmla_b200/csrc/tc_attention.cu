@@ -81,6 +81,7 @@ struct AttnParams {
   int dense;             // 1 for the per-head dense layer
   int64_t nq;            // query tokens per batch element
   int head_major;        // tiles are 128 tokens of one head (dense and fused layers)
+  int64_t tok0;          // head-major: query row r is token tok0 + r of the call (a token range)
   FrameGeom g;
   float scale_log2;      // softmax_scale * log2(e)
   void* out;
@@ -178,8 +179,9 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   const int kv_h = p.dense ? h : 0;                            // head coordinate of the KV maps
   const int tok_div = p.head_major ? 1 : p.heads;              // query row -> token
   const int last_row = min(row0 + kBlockM, p.rows_per_b) - 1;
-  const int64_t kend_first = key_end_rows(p.g, row0 / tok_div);
-  const int64_t kend_last = key_end_rows(p.g, last_row / tok_div);
+  const int64_t tok_base = p.head_major ? p.tok0 : 0;
+  const int64_t kend_first = key_end_rows(p.g, tok_base + row0 / tok_div);
+  const int64_t kend_last = key_end_rows(p.g, tok_base + last_row / tok_div);
   const int n_kv = (int)((kend_last + BN - 1) / BN);
 
   if (threadIdx.x == 0) {
@@ -383,7 +385,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const int r = threadIdx.x;                      // 0..127
     const int row = row0 + r;
     const bool row_valid = row < p.rows_per_b;
-    const int64_t kend = row_valid ? key_end_rows(p.g, row / tok_div) : kend_last;
+    const int64_t kend = row_valid ? key_end_rows(p.g, tok_base + row / tok_div) : kend_last;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     int64_t orow;                                   // this row's index in [rows of q / out / lse]
     if (p.head_major) orow = (((int64_t)b * p.nq + row) * p.heads + h);
@@ -442,8 +444,9 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 #pragma unroll
           for (int t = 0; t < 32; ++t) v[t] = 0.f;
         }
-        const int64_t f = p.g.first_frame + row / p.g.tokens_per_frame;
-        const int rr = row % p.g.tokens_per_frame;
+        const int64_t tok = tok_base + row;
+        const int64_t f = p.g.first_frame + tok / p.g.tokens_per_frame;
+        const int rr = (int)(tok % p.g.tokens_per_frame);
         const int ri = rr / p.g.grid_w, rj = rr % p.g.grid_w;
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
@@ -797,11 +800,11 @@ vmla_status tc_check_fused_attention(const vmla_config& c) {
   return VMLA_OK;
 }
 
-cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t nq, const void* q_nope,
-                                      const void* q_rope, const void* w_uk, const void* w_uv, const void* c,
-                                      const void* k_r, int64_t cap, int64_t valid_rows, const FrameGeom& g,
-                                      const RopeTable& rt, float scale, void* out, float* lse, int* status,
-                                      cudaStream_t st) {
+cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t tok0, int64_t nq,
+                                      const void* q_nope, const void* q_rope, const void* w_uk, const void* w_uv,
+                                      const void* c, const void* k_r, int64_t cap, int64_t valid_rows,
+                                      const FrameGeom& g, const RopeTable& rt, float scale, void* out, float* lse,
+                                      int* status, cudaStream_t st) {
   const int H = cfg.n_heads, dn = cfg.d_nope, dc = cfg.d_c, dv = cfg.d_v;
   TmaMaps5 m{};
   cudaError_t e;
@@ -827,6 +830,7 @@ cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t
   p.heads = H;
   p.dense = 0;
   p.head_major = 1;
+  p.tok0 = tok0;
   p.nq = nq;
   p.g = g;
   p.scale_log2 = scale * 1.4426950408889634f;

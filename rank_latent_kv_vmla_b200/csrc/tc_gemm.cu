@@ -85,11 +85,13 @@ struct RopeLookup {
     }
   }
 
-  // fill the table (all threads of the CTA), then __syncthreads()
-  __device__ void build(float2* smem_tab) const {
+  // fill the table with threads t0 .. t0 + nthreads - 1 (the caller synchronises them afterwards).  The
+  // angle is reduced to [-pi, pi] in double precision, then the MUFU sine / cosine (absolute error
+  // about 1e-6 there, far below the bf16 rounding of the rotated values) keep the build short.
+  __device__ void build(float2* smem_tab, int t0, int nthreads) const {
     const double two_pi = 6.283185307179586476925286766559;
     const double inv_two_pi = 0.15915494309189533576888376337251;
-    for (int e = threadIdx.x; e < n_entries; e += blockDim.x) {
+    for (int e = t0; e < n_entries; e += nthreads) {
       int p = 0;
       while (p + 1 < rt.n_pairs && off[p + 1] <= e) ++p;
       const int64_t v = e - off[p];
@@ -97,7 +99,7 @@ struct RopeLookup {
       double ang = pos * rt.inv_freq[p];
       ang = fma(-two_pi, rint(ang * inv_two_pi), ang);
       float sn, cs;
-      sincosf((float)ang, &sn, &cs);
+      __sincosf((float)ang, &sn, &cs);
       smem_tab[e] = make_float2(cs, sn);
     }
   }
@@ -119,20 +121,26 @@ RopeLookup make_rope_lookup(const RopeTable& rt, const FrameGeom& g, int frames)
 }
 
 // ---- epilogues: called per (row m, 32-column chunk starting at col0) with the fp32 values ----
+// Row m of the GEMM is token tok0 + m % ntok of batch element m / ntok; its c and k^R rows go to the
+// ring of every destination cache (several when replicas of the cache live on other GPUs: plain stores
+// through peer mappings, so the exchange of the chunk's latents is done by this epilogue).
 struct EpiCompress {
   static constexpr bool kRope = true;
-  bf16* c; bf16* k_r; int d_c, d_rope; int64_t ntok, cap; FrameGeom g; RopeLookup rope;
+  bf16* c[kMaxCacheDst]; bf16* k_r[kMaxCacheDst]; int n_dst;
+  int d_c, d_rope; int64_t ntok, tok0, cap; FrameGeom g; RopeLookup rope;
   __device__ void operator()(const float2* tab, int, int64_t m, int col0, float* v) const {
-    const int64_t b = m / ntok, tok = m % ntok;
+    const int64_t b = m / ntok, tok = tok0 + m % ntok;
     const int64_t row = b * cap + ring_row(g, tok);
     if (col0 < d_c) {
-      store32(c + row * d_c + col0, v);
+      for (int d = 0; d < n_dst; ++d) store32(c[d] + row * d_c + col0, v);
     } else {
       const int64_t f = g.first_frame + tok / g.tokens_per_frame;
       const int64_t r = tok % g.tokens_per_frame;
       rope.rotate32(tab, (col0 - d_c) / 2, f, r / g.grid_w, r % g.grid_w, v);
-      store32(k_r + row * d_rope + (col0 - d_c), v);
+      for (int d = 0; d < n_dst; ++d) store32(k_r[d] + row * d_rope + (col0 - d_c), v);
     }
+    // stores to other GPUs' memory: make them visible system-wide before this thread goes on
+    if (n_dst > 1) __threadfence_system();
   }
   __device__ void finish(const float2*, int, int64_t) const {}
 };
@@ -261,7 +269,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
     tmem_alloc(tmem_slot, PL::kTmemCols);
     tmem_relinquish();
   }
-  if constexpr (Epi::kRope) epi.rope.build(rope_tab);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -339,6 +346,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
     }
   } else {
     // ================= epilogue: warps 2..5, TMEM lane quadrant = warp % 4 =================
+    // the RoPE table is built by these four warps while the producer and the MMA warp already run
+    if constexpr (Epi::kRope) {
+      epi.rope.build(rope_tab, threadIdx.x - 64, 128);
+      named_bar_sync(1, 128);
+    }
     const int quad = warp & 3;
     const int r = quad * 32 + (threadIdx.x & 31);
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
@@ -478,7 +490,15 @@ static bool bn_supported(int bn, bool mn_major) {
 cudaError_t tc_compress_append(const vmla_config& cfg, int batch, const void* x, const void* w,
                                const FrameGeom& g, const RopeTable& rt, void* c, void* k_r,
                                cudaStream_t st) {
-  const int64_t ntok = (int64_t)cfg.chunk_frames * cfg.grid_h * cfg.grid_w;
+  CacheDst d{c, k_r};
+  return tc_compress_rows(cfg, batch, 0, (int64_t)cfg.chunk_frames * cfg.grid_h * cfg.grid_w, x, w, g, rt,
+                          &d, 1, st);
+}
+
+cudaError_t tc_compress_rows(const vmla_config& cfg, int batch, int64_t tok0, int64_t ntok, const void* x,
+                             const void* w, const FrameGeom& g, const RopeTable& rt, const CacheDst* dst,
+                             int n_dst, cudaStream_t st) {
+  if (n_dst < 1 || n_dst > kMaxCacheDst) return cudaErrorInvalidValue;
   const int64_t M = batch * ntok;
   const int N = cfg.d_c + cfg.d_rope, K = cfg.dim;
   // one 224-wide column tile per 128 rows leaves most SMs idle at small batch: narrow the column tile
@@ -496,8 +516,19 @@ cudaError_t tc_compress_append(const vmla_config& cfg, int batch, const void* x,
   if ((e = make_map_4d(&mb, w, K, N, 1, 1, (int64_t)K * 2, (int64_t)N * K * 2, (int64_t)N * K * 2, kBK, bn, 1, 128)) != cudaSuccess)
     return e;
   GemmShape sh{M, N, K, 0, wait_limit_ns(), device_status_ptr()};
-  EpiCompress epi{(bf16*)c, (bf16*)k_r, cfg.d_c, cfg.d_rope, ntok, (int64_t)cfg.window_frames * cfg.grid_h * cfg.grid_w, g,
-                  make_rope_lookup(rt, g, cfg.chunk_frames)};
+  EpiCompress epi{};
+  for (int d = 0; d < n_dst; ++d) {
+    epi.c[d] = (bf16*)dst[d].c;
+    epi.k_r[d] = (bf16*)dst[d].k_r;
+  }
+  epi.n_dst = n_dst;
+  epi.d_c = cfg.d_c;
+  epi.d_rope = cfg.d_rope;
+  epi.ntok = ntok;
+  epi.tok0 = tok0;
+  epi.cap = (int64_t)cfg.window_frames * cfg.grid_h * cfg.grid_w;
+  epi.g = g;
+  epi.rope = make_rope_lookup(rt, g, cfg.chunk_frames);
   return dispatch_bn<false>(bn, ma, mb, sh, 1, epi, st);
 }
 

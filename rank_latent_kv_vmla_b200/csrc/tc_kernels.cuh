@@ -9,7 +9,18 @@ namespace vmla {
 // Reason text of the last tc_check_* refusal (thread-local).
 const char* tc_last_reason();
 
+// One destination cache (its c and k_r planes) of a compress call.
+struct CacheDst {
+  void* c;
+  void* k_r;
+};
+constexpr int kMaxCacheDst = 8;
+
 vmla_status tc_check_compress(const vmla_config& cfg);
+// Tokens tok0 .. tok0+ntok-1 of the chunk (x [batch, ntok, dim]) into the rings of n_dst caches.
+cudaError_t tc_compress_rows(const vmla_config& cfg, int batch, int64_t tok0, int64_t ntok, const void* x,
+                             const void* w, const FrameGeom& g, const RopeTable& rt, const CacheDst* dst,
+                             int n_dst, cudaStream_t st);
 cudaError_t tc_compress_append(const vmla_config& cfg, int batch, const void* x, const void* w,
                                const FrameGeom& g, const RopeTable& rt, void* c, void* k_r,
                                cudaStream_t st);
@@ -28,11 +39,12 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
 // Absorbed query, latent attention and value up-projection in one kernel (q_abs and the latent
 // output stay on chip): q_nope [B, Nq, H, d_nope], q_rope [B, Nq, H, 32] -> out [B, Nq, H, d_v].
 vmla_status tc_check_fused_attention(const vmla_config& cfg);
-cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t nq, const void* q_nope,
-                                      const void* q_rope, const void* w_uk, const void* w_uv, const void* c,
-                                      const void* k_r, int64_t cap, int64_t valid_rows, const FrameGeom& g,
-                                      const RopeTable& rt, float scale, void* out, float* lse, int* status,
-                                      cudaStream_t st);
+// tok0: the nq query tokens are tokens tok0 .. tok0+nq-1 of the call (positions and the window rule).
+cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t tok0, int64_t nq,
+                                      const void* q_nope, const void* q_rope, const void* w_uk, const void* w_uv,
+                                      const void* c, const void* k_r, int64_t cap, int64_t valid_rows,
+                                      const FrameGeom& g, const RopeTable& rt, float scale, void* out, float* lse,
+                                      int* status, cudaStream_t st);
 
 vmla_status tc_check_value_up(const vmla_config& cfg);
 cudaError_t tc_value_up(const vmla_config& cfg, int batch, int64_t n_tokens, const void* o_lat,

@@ -260,6 +260,42 @@ vmla_status vmla_compress_append(const vmla_config* cfg, const void* x, const vo
   return VMLA_OK;
 }
 
+vmla_status vmla_compress_append_rows(const vmla_config* cfg, const void* x_rows, const void* w_dkv_kr,
+                                      int64_t first_frame, int64_t token_begin, int64_t n_tokens,
+                                      const vmla_cache* replicas, int32_t n_replicas, void* stream) {
+  vmla_status s = check_config(cfg);
+  if (s != VMLA_OK) return s;
+  VMLA_CHECK_PTR(x_rows);
+  VMLA_CHECK_PTR(w_dkv_kr);
+  if (!replicas || n_replicas < 1 || n_replicas > kMaxCacheDst)
+    return fail(VMLA_ERR_INVALID_ARG, "n_replicas must be in [1, %d]", kMaxCacheDst);
+  if (cfg->dtype != VMLA_BF16) return fail(VMLA_ERR_UNSUPPORTED, "row-range compress runs on the bf16 path only");
+  const int64_t ntok_chunk = (int64_t)cfg->chunk_frames * cfg->grid_h * cfg->grid_w;
+  if (token_begin < 0 || n_tokens <= 0 || token_begin + n_tokens > ntok_chunk)
+    return fail(VMLA_ERR_INVALID_ARG, "token range [%lld, %lld) outside the chunk's %lld tokens",
+                (long long)token_begin, (long long)(token_begin + n_tokens), (long long)ntok_chunk);
+  CacheDst dst[kMaxCacheDst];
+  for (int r = 0; r < n_replicas; ++r) {
+    const vmla_cache& c = replicas[r];
+    if (!c.c || !c.k_r) return fail(VMLA_ERR_INVALID_ARG, "replica %d has a NULL plane", r);
+    if (!aligned16(c.c) || !aligned16(c.k_r)) return fail(VMLA_ERR_MISALIGNED, "replica %d is not 16-byte aligned", r);
+    if (c.batch != replicas[0].batch || c.batch <= 0)
+      return fail(VMLA_ERR_INVALID_ARG, "replicas must share one batch size >= 1");
+    if (c.frames_written != first_frame)
+      return fail(VMLA_ERR_INVALID_ARG, "first_frame %lld does not follow replica %d's frames_written %lld",
+                  (long long)first_frame, r, (long long)c.frames_written);
+    dst[r] = CacheDst{c.c, c.k_r};
+  }
+  s = tc_check_compress(*cfg);
+  if (s != VMLA_OK) return fail(s, "%s", tc_last_reason());
+  const FrameGeom g = make_geom(*cfg, first_frame);
+  const RopeTable rt = make_rope_table(*cfg);
+  cudaError_t e = tc_compress_rows(*cfg, replicas[0].batch, token_begin, n_tokens, x_rows, w_dkv_kr, g, rt, dst,
+                                   n_replicas, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "compress_append_rows launch");
+  return VMLA_OK;
+}
+
 vmla_status vmla_compress_rewrite(const vmla_config* cfg, const void* x, const void* w_dkv_kr,
                                   vmla_cache* cache, void* stream) {
   vmla_status s = check_compress_args(cfg, x, w_dkv_kr, cache);
@@ -369,10 +405,50 @@ vmla_status vmla_latent_attention_fused(const vmla_config* cfg, const void* q_no
   const int64_t cap = (int64_t)cfg->window_frames * T_f;
   const int64_t valid_rows =
       (cache->frames_written < cfg->window_frames ? cache->frames_written : cfg->window_frames) * T_f;
-  cudaError_t e = tc_latent_attention_fused(*cfg, cache->batch, nq, q_nope, q_rope, w_uk, w_uv, cache->c,
+  cudaError_t e = tc_latent_attention_fused(*cfg, cache->batch, 0, nq, q_nope, q_rope, w_uk, w_uv, cache->c,
                                             cache->k_r, cap, valid_rows, g, rt, softmax_scale(*cfg), out,
                                             lse, device_status_ptr(), as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "latent_attention_fused launch");
+  return VMLA_OK;
+}
+
+vmla_status vmla_latent_attention_fused_rows(const vmla_config* cfg, const void* q_nope, const void* q_rope,
+                                             const void* w_uk, const void* w_uv, const vmla_cache* cache,
+                                             int64_t first_frame, int32_t n_query_chunks, int64_t token_begin,
+                                             int64_t n_tokens, void* out, float* lse, void* stream) {
+  vmla_status s = check_config(cfg);
+  if (s != VMLA_OK) return s;
+  if (!cache) return fail(VMLA_ERR_INVALID_ARG, "cache is NULL");
+  VMLA_CHECK_PTR(q_nope);
+  VMLA_CHECK_PTR(q_rope);
+  VMLA_CHECK_PTR(w_uk);
+  VMLA_CHECK_PTR(w_uv);
+  VMLA_CHECK_PTR(cache->c);
+  VMLA_CHECK_PTR(cache->k_r);
+  VMLA_CHECK_PTR(out);
+  if (lse && !aligned16(lse)) return fail(VMLA_ERR_MISALIGNED, "lse is not 16-byte aligned");
+  if (cache->batch <= 0) return fail(VMLA_ERR_INVALID_ARG, "cache->batch must be >= 1");
+  if (cfg->dtype != VMLA_BF16)
+    return fail(VMLA_ERR_UNSUPPORTED, "the fused call runs on the bf16 tensor-core path only");
+  s = check_window(*cfg, cache->frames_written, first_frame, n_query_chunks);
+  if (s != VMLA_OK) return s;
+  const int64_t T_f = (int64_t)cfg->grid_h * cfg->grid_w;
+  const int64_t nq_call = (int64_t)n_query_chunks * cfg->chunk_frames * T_f;
+  if (token_begin < 0 || n_tokens <= 0 || token_begin + n_tokens > nq_call)
+    return fail(VMLA_ERR_INVALID_ARG, "token range [%lld, %lld) outside the call's %lld query tokens",
+                (long long)token_begin, (long long)(token_begin + n_tokens), (long long)nq_call);
+  s = tc_check_fused_attention(*cfg);
+  if (s != VMLA_OK) return fail(s, "%s", tc_last_reason());
+  const FrameGeom g = make_geom(*cfg, first_frame);
+  const RopeTable rt = make_rope_table(*cfg);
+  const int64_t cap = (int64_t)cfg->window_frames * T_f;
+  const int64_t valid_rows =
+      (cache->frames_written < cfg->window_frames ? cache->frames_written : cfg->window_frames) * T_f;
+  cudaError_t e = tc_latent_attention_fused(*cfg, cache->batch, token_begin, n_tokens, q_nope, q_rope, w_uk,
+                                            w_uv, cache->c, cache->k_r, cap, valid_rows, g, rt,
+                                            softmax_scale(*cfg), out, lse, device_status_ptr(),
+                                            as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "latent_attention_fused_rows launch");
   return VMLA_OK;
 }
 

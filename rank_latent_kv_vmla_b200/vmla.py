@@ -26,7 +26,9 @@ EXPORTED = ("vmla_compress_append", "vmla_absorb_q", "vmla_latent_attention", "v
             "vmla_status_string", "vmla_last_error_detail", "vmla_abi_version",
             "vmla_compress_rewrite", "vmla_dense_rewrite", "vmla_plan_capacity",
             "vmla_latent_attention_fused", "vmla_executor_workspace_bytes", "vmla_executor_create",
-            "vmla_executor_submit", "vmla_executor_wait", "vmla_executor_destroy")
+            "vmla_executor_submit", "vmla_executor_wait", "vmla_executor_destroy",
+            "vmla_compress_append_rows", "vmla_latent_attention_fused_rows", "vmla_ipc_export",
+            "vmla_ipc_import", "vmla_ipc_release")
 
 
 class VmlaError(RuntimeError):
@@ -52,6 +54,10 @@ class CCache(ctypes.Structure):
 class CCapacity(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in ("max_batch", "cache_bytes_per_seq",
                                                 "buffer_bytes_per_seq", "weight_bytes")]
+
+
+class CIpcHandle(ctypes.Structure):
+    _fields_ = [("bytes", ctypes.c_ubyte * 64), ("offset", ctypes.c_int64)]
 
 
 class CDenseCache(ctypes.Structure):
@@ -81,6 +87,11 @@ def _load():
         "vmla_plan_capacity": [cfgp, I32, I32, I64, I64, I64, P(CCapacity)],
         "vmla_latent_attention_fused": [cfgp, VP, VP, VP, VP, P(CCache), I64, I32, VP, VP, VP],
         "vmla_executor_create": [cfgp, I32, VP, I64, VP, P(VP)],
+        "vmla_compress_append_rows": [cfgp, VP, VP, I64, I64, I64, P(CCache), I32, VP],
+        "vmla_latent_attention_fused_rows": [cfgp, VP, VP, VP, VP, P(CCache), I64, I32, I64, I64, VP, VP, VP],
+        "vmla_ipc_export": [VP, P(CIpcHandle)],
+        "vmla_ipc_import": [P(CIpcHandle), P(VP)],
+        "vmla_ipc_release": [VP],
         "vmla_executor_submit": [VP, P(CCache), VP, VP, VP, VP, VP, VP, VP],
         "vmla_executor_wait": [VP],
         "vmla_executor_destroy": [VP],
@@ -393,6 +404,59 @@ def plan_capacity(cfg: VmlaConfig, n_layers: int, budget_bytes: int, *, dense: b
     return {n: int(getattr(out, n)) for n, _ in CCapacity._fields_}
 
 
+def compress_append_rows(cfg: VmlaConfig, x_rows: torch.Tensor, w_dkv_kr: torch.Tensor, first_frame: int,
+                         token_begin: int, replicas, batch: int) -> None:
+    """Compress tokens token_begin .. token_begin + n - 1 of the chunk (x_rows [B, n, D]) into the ring of
+    every replica (a sequence of CCache structs, possibly holding peer pointers).  frames_written of the
+    replicas is not advanced."""
+    n = x_rows.shape[1]
+    cc = c_config(cfg)
+    arr = (CCache * len(replicas))(*replicas)
+    check(LIB.vmla_compress_append_rows(ctypes.byref(cc), _arg(x_rows, cfg, (batch, n, cfg.dim), "x_rows"),
+                                        _arg(w_dkv_kr, cfg, (cfg.d_c + cfg.d_rope, cfg.dim), "w_dkv_kr"),
+                                        first_frame, token_begin, n, arr, len(replicas), _stream(x_rows)))
+
+
+def latent_attention_fused_rows(cfg: VmlaConfig, q_nope: torch.Tensor, q_rope: torch.Tensor, w_uk: torch.Tensor,
+                                w_uv: torch.Tensor, cache: LatentCache, first_frame: int, token_begin: int,
+                                n_query_chunks: int = 1, out: Optional[torch.Tensor] = None,
+                                lse: Optional[torch.Tensor] = None, want_lse: bool = False):
+    """The fused attention for query tokens token_begin .. token_begin + n - 1 of the call only:
+    q^nope [B, n, H, d_nope], q^rope [B, n, H, d_rope] -> o [B, n, H, d_v] (and lse [B, n, H])."""
+    B, n, H = cache.batch, q_nope.shape[1], cfg.n_heads
+    if out is None:
+        out = torch.empty((B, n, H, cfg.d_v), dtype=_dtype(cfg), device=q_nope.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n, H), dtype=torch.float32, device=q_nope.device)
+    cc = c_config(cfg)
+    check(LIB.vmla_latent_attention_fused_rows(
+        ctypes.byref(cc), _arg(q_nope, cfg, (B, n, H, cfg.d_nope), "q_nope"),
+        _arg(q_rope, cfg, (B, n, H, cfg.d_rope), "q_rope"), _arg(w_uk, cfg, (H, cfg.d_nope, cfg.d_c), "w_uk"),
+        _arg(w_uv, cfg, (H, cfg.d_v, cfg.d_c), "w_uv"), ctypes.byref(cache.struct), first_frame, n_query_chunks,
+        token_begin, n, _arg(out, cfg, (B, n, H, cfg.d_v), "out"), lse.data_ptr() if lse is not None else None,
+        _stream(q_nope)))
+    return (out, lse) if (lse is not None) else out
+
+
+def ipc_export(t: torch.Tensor) -> bytes:
+    """Serialisable handle (72 bytes) of the device buffer holding tensor t."""
+    h = CIpcHandle()
+    check(LIB.vmla_ipc_export(t.data_ptr(), ctypes.byref(h)))
+    return bytes(ctypes.string_at(ctypes.addressof(h), ctypes.sizeof(h)))
+
+
+def ipc_import(handle: bytes) -> int:
+    """Map another process's buffer (a handle from ipc_export) into this one; returns the device pointer."""
+    h = CIpcHandle.from_buffer_copy(handle)
+    p = ctypes.c_void_p()
+    check(LIB.vmla_ipc_import(ctypes.byref(h), ctypes.byref(p)))
+    return int(p.value)
+
+
+def ipc_release(ptr: int) -> None:
+    check(LIB.vmla_ipc_release(ptr))
+
+
 class Executor:
     """Streaming executor of the C library: layer steps with inputs and outputs in (pinned) host memory,
     the copies of neighbouring steps overlapping each step's kernels.  The device workspace is allocated
@@ -482,4 +546,6 @@ __all__ = ["LIB", "VmlaError", "LatentCache", "DenseCache", "compress_append", "
            "latent_attention", "value_up", "rope_q", "dense_append", "dense_mha", "device_status",
            "launch_count", "latent_cache_bytes", "dense_cache_bytes", "layer_step", "c_config",
            "compress_rewrite", "dense_rewrite", "plan_capacity", "CCapacity", "latent_attention_fused", "Executor",
+           "compress_append_rows", "latent_attention_fused_rows", "ipc_export", "ipc_import", "ipc_release",
+           "CIpcHandle",
            "CConfig", "CCache", "CDenseCache", "EXPORTED", "VMLA_F32", "VMLA_BF16"]
