@@ -121,19 +121,21 @@ def frame_of_slot(slot: int, frames_written: int, window_frames: int) -> int:
 
 
 def ring_from_history(hist: np.ndarray, frames_written: int, window_frames: int,
-                      tokens_per_frame: int) -> tuple:
-    """Expected ring-buffer plane from the full history ``hist`` [frames_written*T_f, d] of one batch
-    element: slot s holds frame frame_of_slot(s).  Returns (plane [W*T_f, d] with NaN in unwritten
-    slots, written-row mask [W*T_f])."""
+                      tokens_per_frame: int, first_frame: int = 0) -> tuple:
+    """Expected ring-buffer plane from the history ``hist`` of one batch element, which holds frames
+    first_frame .. frames_written-1 in order ([(frames_written - first_frame)*T_f, d]): slot s holds frame
+    frame_of_slot(s); frames before first_frame were never written.  Returns (plane [W*T_f, d] with NaN
+    in unwritten slots, written-row mask [W*T_f])."""
     d = hist.shape[-1]
     plane = np.full((window_frames * tokens_per_frame, d), np.nan, dtype=F64)
     written = np.zeros(window_frames * tokens_per_frame, dtype=bool)
     for s in range(window_frames):
         f = frame_of_slot(s, frames_written, window_frames)
-        if f < 0:
+        if f < first_frame:
             continue
+        r = f - first_frame
         plane[s * tokens_per_frame:(s + 1) * tokens_per_frame] = \
-            hist[f * tokens_per_frame:(f + 1) * tokens_per_frame]
+            hist[r * tokens_per_frame:(r + 1) * tokens_per_frame]
         written[s * tokens_per_frame:(s + 1) * tokens_per_frame] = True
     return plane, written
 

@@ -71,9 +71,12 @@ class OracleLayer:
         self.w_uv = f64(inp.w_uv)
         self.hist = [O.History(cfg.d_c, cfg.d_rope) for _ in range(batch)]
         self.frames_written = 0
+        self.first_frame = None          # absolute frame of the first append (histories may start late)
 
     def append(self, x: torch.Tensor):
         cfg = self.cfg
+        if self.first_frame is None:
+            self.first_frame = self.frames_written
         pos = O.token_positions(self.frames_written, cfg.chunk_tokens, cfg.grid_h, cfg.grid_w)
         xs = f64(x)
         for b in range(self.batch):
@@ -93,10 +96,11 @@ class OracleLayer:
 
     def ring(self, b: int):
         cfg = self.cfg
+        f0 = self.first_frame or 0
         c, written = O.ring_from_history(self.hist[b].c, self.frames_written, cfg.window_frames,
-                                         cfg.tokens_per_frame)
+                                         cfg.tokens_per_frame, first_frame=f0)
         k_r, _ = O.ring_from_history(self.hist[b].k_r, self.frames_written, cfg.window_frames,
-                                     cfg.tokens_per_frame)
+                                     cfg.tokens_per_frame, first_frame=f0)
         return c, k_r, written
 
     def q_abs(self, q_nope: torch.Tensor, q_rope: torch.Tensor, first_frame: int):

@@ -184,6 +184,18 @@ def test_ring_matches_explicit_ring_writes():
     assert [O.frame_of_slot(s, 6, W) for s in range(W)] == [3, 4, 5]
     assert [O.frame_of_slot(s, 2, W) for s in range(W)] == [0, 1, -1]
     assert O.frame_of_slot(0, 0, W) == -1
+    # a history that starts at a late absolute frame F0: the same explicit ring, slots by f mod W
+    F0 = 1_000_004
+    ring = np.full((W * T, d), np.nan)
+    for fw in range(F0 + 1, F0 + 6):
+        f = fw - 1
+        s = f % W
+        r = f - F0
+        ring[s * T:(s + 1) * T] = hist[r * T:(r + 1) * T]
+        plane, written = O.ring_from_history(hist[:(fw - F0) * T], fw, W, T, first_frame=F0)
+        np.testing.assert_array_equal(np.isnan(plane[:, 0]), np.isnan(ring[:, 0]))
+        np.testing.assert_array_equal(plane[written], ring[written])
+        assert written.sum() == min(fw - F0, W) * T
 
 
 def test_window_mask_matches_streaming_simulation():
