@@ -838,7 +838,7 @@ cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t
   p.lse = lse;
   p.status = status;
   p.limit_ns = wait_limit_ns();
-  p.drop_kv_tile = -1;
+  p.drop_kv_tile = take_drop_kv_tile();
   p.q_rope = q_rope;
   p.d_nope = dn;
   p.d_v = dv;

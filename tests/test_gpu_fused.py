@@ -141,3 +141,36 @@ def test_wan_fused_full_size_sampled(V):
         assert_close(f64(lse[b][rows]), ref["lse"], cfg, f"lse b{b}")
         rel_l2, max_rel = errors(f64(o[b]), f64(o3[b]))
         assert rel_l2 <= 2e-3, (b, max_rel, rel_l2)
+
+
+def test_fused_bounded_wait_reports_timeout_and_context_survives(V):
+    """A KV tile the fused kernel never loads: the bounded wait runs out, every role winds down (the
+    up-projection weights are not loaded, no output is written), vmla_device_status reports the code,
+    and the next fused call on the same context is correct."""
+    cfg = MID
+    inp = synthetic.draw_layer(cfg, batch=1, seed=3600, n_chunks=3)
+    cache = V.LatentCache(cfg, 1, device=DEV)
+    for x in inp.x_chunks:
+        f0 = cache.frames_written
+        V.compress_append(cfg, _to(x), _to(inp.w_dkv_kr), cache)
+    args = (_to(inp.q_nope), _to(inp.q_rope), _to(inp.w_uk), _to(inp.w_uv))
+    torch.cuda.synchronize()
+    assert V.device_status() == 0
+    old = V.set_wait_timeout_ms(20)
+    try:
+        V.debug_drop_kv_tile(1)
+        V.latent_attention_fused(cfg, *args, cache, f0)
+        torch.cuda.synchronize()
+        assert V.device_status() != 0
+        assert V.device_status() == 0          # reading clears it
+    finally:
+        V.debug_drop_kv_tile(-1)
+        V.set_wait_timeout_ms(old)
+    o = V.latent_attention_fused(cfg, *args, cache, f0)
+    torch.cuda.synchronize()
+    assert V.device_status() == 0
+    orc = OracleLayer(cfg, inp, 1)
+    for x in inp.x_chunks:
+        orc.append(x)
+    ref = orc.reference(0, inp.q_nope, inp.q_rope, f0)
+    assert_close(f64(o[0]), ref["o"], cfg, "fused o after a timed-out launch")
