@@ -6,10 +6,13 @@ rows against the full 21-frame window (32760 cached tokens), and the value up-pr
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B] [--impl reference]
 
-Prints one JSON line (rank 0).  ``value`` is latent-attention TFLOP/s (2*B*H*Nq*Nk*(2*d_c + d_rope)
-algorithmic flops per step, whole step timed on the device with CUDA events, L2 flushed between
-steps), summed over ranks (each rank runs its own batch: weak scaling).  ``--impl reference`` times
-the float64 CPU oracle on a bounded sample of the same workload instead.
+Prints one JSON line (rank 0).  ``value`` is latent-attention TFLOP/s: 2*B*H*Nq*Nk*(2*d_c + d_rope)
+algorithmic flops per step, the whole step timed on the device with CUDA events, summed over ranks
+(each rank runs its own batch: weak scaling).  No step finds the previous one's data in L2:
+- by default consecutive steps cycle over 10 layer caches and 4 input sets, 262 MB at B = 1, more
+  than the 126 MB L2, as consecutive layers of a rollout do;
+- with ``--l2 flush`` one cache is used, with a 512 MB write between steps.
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the same workload instead.
 """
 from __future__ import annotations
 
@@ -51,6 +54,10 @@ def parse():
                     help="batch: each rank runs its own sequences (weak scaling, no collective); query: one "
                          "batch whose chunk query rows are sharded over the ranks, each holding a replica of "
                          "the latent cache that every rank's compress kernel writes (strong scaling)")
+    ap.add_argument("--l2", default="rotate", choices=["rotate", "flush"],
+                    help="rotate: consecutive steps use different layer caches (10 x 14.7 MB at B = 1) and input "
+                         "sets, more than L2, as consecutive layers of a rollout do; flush: one cache, and a "
+                         "512 MB write between steps")
     ap.add_argument("--path", default="fused", choices=["fused", "three"],
                     help="fused: compress + one fused attention launch per step; three: compress + "
                          "absorb + attention + value-up launches (the other path is timed beside it)")
@@ -632,14 +639,25 @@ def main():
     w_uk, w_uv = inp.w_uk.to(dev), inp.w_uv.to(dev)
     xs = [x.to(dev) for x in inp.x_chunks[prefill:]]
     qs = [(qn.to(dev), qr.to(dev)) for qn, qr in extra_q]
-    cache = V.LatentCache(cfg, B, device=dev)
-    for x in inp.x_chunks[:prefill]:
-        V.compress_append(cfg, x.to(dev), w, cache)
+    # the layer caches the steps cycle over: E2E_LAYERS of them (147 MB at B = 1, with the 115 MB of input
+    # sets more than L2, so no step finds the previous step's data in L2), or one with --l2 flush
+    rotate = args.l2 == "rotate"
+    caches = []
+    for _ in range(E2E_LAYERS if rotate else 1):
+        c1 = V.LatentCache(cfg, B, device=dev)
+        for x in inp.x_chunks[:prefill]:
+            V.compress_append(cfg, x.to(dev), w, c1)
+        caches.append(c1)
+    cache = caches[0]
     bufs = {"q_abs": torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_qk), dtype=torch.bfloat16, device=dev),
             "o_latent": torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_c), dtype=torch.bfloat16, device=dev),
             "o": torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)}
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = None if rotate else torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+
+    def between_steps():
+        if flush is not None:
+            flush.zero_()
 
     fused = args.path == "fused"
     names = (["compress_append", "latent_attention_fused"] if fused else
@@ -650,6 +668,7 @@ def main():
         x = xs[i % N_INPUT_SETS] if x is None else x
         if qn is None:
             qn, qr = qs[i % N_INPUT_SETS]
+        cache = caches[i % len(caches)]
         f0 = cache.frames_written
         if ev: ev[0].record(stream)
         V.compress_append(cfg, x, w, cache, f0)
@@ -667,7 +686,7 @@ def main():
 
     for i in range(args.warmup):
         step(i)
-        flush.zero_()
+        between_steps()
     torch.cuda.synchronize()
     assert V.device_status() == 0
 
@@ -680,7 +699,7 @@ def main():
     wall0 = time.perf_counter()
     for i in range(args.steps):
         step(args.warmup + i, evs[i])
-        flush.zero_()
+        between_steps()
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
     launches = V.launch_count() - launches0
@@ -721,7 +740,7 @@ def main():
     for i in range(2 * ab_steps):
         use = (i % 4) in (0, 3)                   # fused, three, three, fused, ...
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        flush.zero_()
+        between_steps()
         a.record(stream)
         step(args.warmup + args.steps + i, use_fused=use)
         b.record(stream)
@@ -736,8 +755,8 @@ def main():
     # overlaps each step's host -> device and device -> host copies with the neighbouring steps'
     # kernels.  Steps cycle over E2E_LAYERS layer caches (147 MB with the inputs' staging: more than
     # L2, so no flush is needed between steps) ----
-    e_caches = [cache]
-    for _ in range(E2E_LAYERS - 1):
+    e_caches = list(caches)
+    while len(e_caches) < E2E_LAYERS:
         c2 = V.LatentCache(cfg, B, device=dev)
         for x in inp.x_chunks[:prefill]:
             V.compress_append(cfg, x.to(dev), w, c2)
@@ -790,12 +809,13 @@ def main():
             V.dense_mha(cfg, dq, dcache, f0, out=do)
             ev[3].record(stream)
 
+        # the dense cache (201 MB per sequence) alone exceeds L2
         for i in range(3):
             dstep(i, devs[0])
-            flush.zero_()
+            between_steps()
         for i in range(dsteps):
             dstep(i, devs[i])
-            flush.zero_()
+            between_steps()
         torch.cuda.synchronize()
         d_step_ms = statistics.mean(devs[i][0].elapsed_time(devs[i][3]) for i in range(dsteps))
         d_mha_ms = statistics.mean(devs[i][2].elapsed_time(devs[i][3]) for i in range(dsteps))
@@ -822,7 +842,11 @@ def main():
                            "query_tokens": cfg.chunk_tokens, "cached_tokens": cfg.window_tokens,
                            "heads": cfg.n_heads, "d_c": cfg.d_c, "d_rope": cfg.d_rope, "d_v": cfg.d_v,
                            "dim": cfg.dim, "parallelism": f"dp{world} (independent sequences)",
-                           "l2": "flushed between steps (512 MB write)",
+                           "l2": ("inputs larger than L2: steps cycle over %d layer caches (%.0f MB) and %d input "
+                                  "sets (%.0f MB)" % (len(caches), len(caches) * V.latent_cache_bytes(cfg, B) / 1e6,
+                                                      N_INPUT_SETS, N_INPUT_SETS * 2 * (xs[0].numel() + qs[0][0].numel() +
+                                                                                     qs[0][1].numel()) / 1e6)
+                                  if rotate else "flushed between steps (512 MB write)"),
                            "path": ("compress + fused absorb/attention/value-up" if fused
                                     else "compress + absorb + attention + value-up")},
                 "query_tokens_per_s": q_tok_s,
