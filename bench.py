@@ -121,12 +121,18 @@ def traffic_for(kernel: str, source_hash: str):
 
 
 def source_hash(names):
+    """Hash of the kernel sources' code: comments and blank space removed, so that only a change of
+    the code itself marks a recorded ncu traffic figure as stale."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for n in names:
         p = os.path.join(ROOT, "rank_latent_kv_vmla_b200", "csrc", n)
         if os.path.exists(p):
-            h.update(open(p, "rb").read())
+            text = open(p, encoding="utf-8").read()
+            text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)      # block comments
+            text = re.sub(r"//[^\n]*", " ", text)                     # line comments
+            h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

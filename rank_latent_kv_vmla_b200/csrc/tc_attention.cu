@@ -12,14 +12,15 @@
 //               O += P_{j-1} V_{j-1} with P read from TMEM (it overwrites S_{j-1} as bf16);
 //   warps 0-3   one thread per query row (= TMEM lane): first the Q row into TMEM (when Q is kept
 //               in TMEM), then per tile the softmax: masked running max with a lazy rescale of O (only
-//               when the max grows by more than 2^8), exp2, row sum, P to TMEM; finally O / l to
-//               global memory and the log-sum-exp.  The softmax is issue-bound, so it uses 3-input
-//               max and packed f32x2 FMA / add instructions.
-// Keeping Q in TMEM makes S = Q K^T read only K from shared memory: with Q re-read from shared
-// memory by every MMA, the QK^T MMAs, the P V MMAs and the TMA writes together exceed the shared
-// memory bandwidth and the tensor pipe stalls.  The TMEM budget (512 columns: 2 S buffers, O, Q) then
-// sets BN: 96 keys for d_c = 192, 128 keys for smaller latents and for the dense layer.
-// The KV ring is released by tcgen05.commit after the P V MMAs that last read a stage.
+//               when the max grows by more than 2^8), exp2 (a quarter of them by an FMA-pipe
+//               polynomial), row sum, P to TMEM in two key halves, each released to the P V MMAs by
+//               its own barrier; finally O / l to global memory and the log-sum-exp.  The softmax is
+//               latency-bound with one warp per SM sub-partition, so it uses 3-input max and packed
+//               f32x2 FMA / add instructions.
+// Q lives in TMEM (S = Q K^T then reads only K from shared memory) where the TMEM budget allows it
+// with 128-key tiles: d_c = 64 / 128 and the dense layer.  For d_c = 192 / 256 (2 S buffers + O leave
+// no room for Q at 128 keys) Q stays in shared memory; a Q-in-TMEM build with 96-key tiles was
+// measured slower.  The KV ring is released by tcgen05.commit after the P V MMAs that last read a stage.
 //
 // The fused latent instance also does the two per-head projections around the attention (the
 // technical summary's Method item 2: keys and values are rebuilt from the latent with the per-head
