@@ -477,6 +477,15 @@ def run_workload(args):
                    "query_tokens_per_s": B * cfg.chunk_tokens / (ms * 1e-3),
                    "cache_bytes_per_layer": V.latent_cache_bytes(cfg, B),
                    "cache_fraction_of_dense": V.latent_cache_bytes(cfg, B) / V.dense_cache_bytes(cfg, B)}
+            if d_c >= 128:
+                # the fused call: absorb + attention + value-up in one launch (what the layer step runs)
+                wuv = inp.w_uv.to(dev)
+                o_f = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
+                for _ in range(3):
+                    V.latent_attention_fused(cfg, qn, qr, wuk, wuv, cache, f0, out=o_f)
+                fms = _time(lambda: V.latent_attention_fused(cfg, qn, qr, wuk, wuv, cache, f0, out=o_f), 20, stream)
+                row.update({"fused_ms": fms, "fused_attention_tflops": attention_flops(cfg, B) / (fms * 1e-3) / 1e12})
+                ms = fms
             if args.workload == "batch8":
                 w_kv = synthetic.draw_dense_weights(cfg, 77).to(dev)
                 dcache = V.DenseCache(cfg, B, device=dev)
@@ -489,6 +498,7 @@ def run_workload(args):
                 dms = _time(lambda: V.dense_mha(cfg, q, dcache, f0, out=o_d), 20, stream)
                 row.update({"dense_mha_ms": dms, "dense_tflops": dense_attention_flops(cfg, B) / (dms * 1e-3) / 1e12,
                             "attention_time_ratio_latent_over_dense": ms / dms,
+                            "ratio_uses": "fused call (absorb + attention + value-up) vs dense MHA",
                             "dense_cache_bytes_per_layer": V.dense_cache_bytes(cfg, B)})
                 del dcache
             rows.append(row)

@@ -210,3 +210,34 @@ def test_executor_workspace_and_rejections():
     assert st == V.VMLA_ERR_INVALID_ARG
     assert V.LIB.vmla_executor_wait(None) == V.VMLA_ERR_INVALID_ARG
     assert V.LIB.vmla_executor_destroy(None) == V.VMLA_OK
+
+
+def test_binding_rejects_host_tensors_and_bad_shapes():
+    """The Python binding checks device, dtype, contiguity and shape before calling the library."""
+    import torch
+    cfg = WAN
+    x = torch.zeros((1, cfg.chunk_tokens, cfg.dim), dtype=torch.bfloat16)           # a host tensor
+    w = torch.zeros((cfg.d_c + cfg.d_rope, cfg.dim), dtype=torch.bfloat16)
+    cache = V.LatentCache(cfg, 1, device="cpu")
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        V.compress_append(cfg, x, w, cache)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        V.compress_rewrite(cfg, x, w, cache)
+    with pytest.raises(ValueError):
+        V.absorb_q(cfg, torch.zeros((1, 7, cfg.n_heads, cfg.d_nope), dtype=torch.bfloat16),
+                   torch.zeros((1, 7, cfg.n_heads, cfg.d_rope), dtype=torch.bfloat16),
+                   torch.zeros((cfg.n_heads, cfg.d_nope, cfg.d_c), dtype=torch.bfloat16), 0)   # 7 tokens
+    with pytest.raises(ValueError):
+        V.latent_attention_fused(cfg, torch.zeros((1, 7, cfg.n_heads, cfg.d_nope), dtype=torch.bfloat16),
+                                 torch.zeros((1, 7, cfg.n_heads, cfg.d_rope), dtype=torch.bfloat16), w, w, cache, 0)
+    assert V.latent_cache_bytes(cfg, 1) == cache.nbytes()
+
+
+def test_status_codes_match_header():
+    text = open(HEADER).read()
+    for name, value in (("VMLA_OK", 0), ("VMLA_ERR_INVALID_ARG", 1), ("VMLA_ERR_UNSUPPORTED", 2),
+                        ("VMLA_ERR_MISALIGNED", 3), ("VMLA_ERR_CUDA", 4), ("VMLA_ERR_TIMEOUT", 5)):
+        assert re.search(r"\b%s\s*=\s*%d\b" % (name, value), text), name
+        assert getattr(V, name) == value
+    for name, value in (("VMLA_PATH_LATENT", 0), ("VMLA_PATH_DENSE", 1), ("VMLA_PATH_LATENT_FUSED", 2)):
+        assert re.search(r"\b%s\s*=\s*%d\b" % (name, value), text), name
