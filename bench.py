@@ -54,6 +54,8 @@ def parse():
                     help="batch: each rank runs its own sequences (weak scaling, no collective); query: one "
                          "batch whose chunk query rows are sharded over the ranks, each holding a replica of "
                          "the latent cache that every rank's compress kernel writes (strong scaling)")
+    ap.add_argument("--nvtx", action="store_true",
+                    help="mark every timed step and each of its calls with an NVTX range (for Nsight Systems)")
     ap.add_argument("--l2", default="rotate", choices=["rotate", "flush"],
                     help="rotate: consecutive steps use different layer caches (10 x 14.7 MB at B = 1) and input "
                          "sets, more than L2, as consecutive layers of a rollout do; flush: one cache, and a "
@@ -680,7 +682,25 @@ def main():
              ["compress_append", "absorb_q", "latent_attention", "value_up"])
     n_ev = len(names) + 1
 
+    nvtx = torch.cuda.nvtx if args.nvtx else None
+
+    def mark(name):
+        if nvtx is not None:
+            nvtx.range_pop()
+            nvtx.range_push(name)
+
     def step(i, ev=None, x=None, qn=None, qr=None, use_fused=fused):
+        if nvtx is not None:
+            nvtx.range_push(f"step {i}")
+            nvtx.range_push("compress_append")
+        try:
+            _step(i, ev, x, qn, qr, use_fused)
+        finally:
+            if nvtx is not None:
+                nvtx.range_pop()
+                nvtx.range_pop()
+
+    def _step(i, ev, x, qn, qr, use_fused):
         x = xs[i % N_INPUT_SETS] if x is None else x
         if qn is None:
             qn, qr = qs[i % N_INPUT_SETS]
@@ -690,13 +710,17 @@ def main():
         V.compress_append(cfg, x, w, cache, f0)
         if ev: ev[1].record(stream)
         if use_fused:
+            mark("latent_attention_fused")
             V.latent_attention_fused(cfg, qn, qr, w_uk, w_uv, cache, f0, out=bufs["o"])
             if ev: ev[2].record(stream)
             return
+        mark("absorb_q")
         V.absorb_q(cfg, qn, qr, w_uk, f0, out=bufs["q_abs"])
         if ev: ev[2].record(stream)
+        mark("latent_attention")
         V.latent_attention(cfg, bufs["q_abs"], cache, f0, out=bufs["o_latent"])
         if ev: ev[3].record(stream)
+        mark("value_up")
         V.value_up(cfg, bufs["o_latent"], w_uv, out=bufs["o"])
         if ev: ev[4].record(stream)
 

@@ -158,6 +158,26 @@ def _arg(t: torch.Tensor, cfg: VmlaConfig, shape, name: str) -> int:
     return t.data_ptr()
 
 
+def _cache_key(cfg: VmlaConfig) -> dict:
+    """The configuration fields a saved cache must match to be restored."""
+    return {n: getattr(cfg, n) for n in ("n_heads", "d_nope", "d_rope", "d_c", "d_v", "grid_h", "grid_w",
+                                          "chunk_frames", "window_frames", "dtype")}
+
+
+def _save_planes(path, kind: str, cfg: VmlaConfig, batch: int, frames_written: int, planes: dict) -> None:
+    torch.save({"kind": kind, "config": _cache_key(cfg), "batch": batch, "frames_written": frames_written,
+                "planes": {k: v.detach().to("cpu") for k, v in planes.items()}}, path)
+
+
+def _load_planes(path, kind: str, cfg: VmlaConfig) -> dict:
+    state = torch.load(path, map_location="cpu", weights_only=True)
+    if state.get("kind") != kind:
+        raise ValueError(f"{path} holds a {state.get('kind')} cache, not a {kind} cache")
+    if state["config"] != _cache_key(cfg):
+        raise ValueError(f"{path} was saved with configuration {state['config']}, not {_cache_key(cfg)}")
+    return state
+
+
 class LatentCache:
     """One layer's latent cache: c [B, W*T_f, d_c] and k_r [B, W*T_f, d_rope] plus frames_written."""
 
@@ -183,6 +203,20 @@ class LatentCache:
     def nbytes(self) -> int:
         return self.c.numel() * self.c.element_size() + self.k_r.numel() * self.k_r.element_size()
 
+    def save(self, path) -> None:
+        """Checkpoint: the ring planes and frames_written (the whole state of the layer's cache)."""
+        _save_planes(path, "latent", self.cfg, self.batch, self.frames_written, {"c": self.c, "k_r": self.k_r})
+
+    @classmethod
+    def load(cls, path, cfg: VmlaConfig, device="cuda") -> "LatentCache":
+        """Restore a checkpoint written by save(); streaming continues exactly where it stopped."""
+        state = _load_planes(path, "latent", cfg)
+        cache = cls(cfg, state["batch"], device=device)
+        cache.c.copy_(state["planes"]["c"])
+        cache.k_r.copy_(state["planes"]["k_r"])
+        cache.struct.frames_written = state["frames_written"]
+        return cache
+
 
 class DenseCache:
     """Dense per-head cache of the comparison layer: k [B, W*T_f, H, d_h], v [B, W*T_f, H, d_v]."""
@@ -204,6 +238,18 @@ class DenseCache:
 
     def nbytes(self) -> int:
         return self.k.numel() * self.k.element_size() + self.v.numel() * self.v.element_size()
+
+    def save(self, path) -> None:
+        _save_planes(path, "dense", self.cfg, self.struct.batch, self.frames_written, {"k": self.k, "v": self.v})
+
+    @classmethod
+    def load(cls, path, cfg: VmlaConfig, device="cuda") -> "DenseCache":
+        state = _load_planes(path, "dense", cfg)
+        cache = cls(cfg, state["batch"], device=device)
+        cache.k.copy_(state["planes"]["k"])
+        cache.v.copy_(state["planes"]["v"])
+        cache.struct.frames_written = state["frames_written"]
+        return cache
 
 
 def compress_append(cfg: VmlaConfig, x: torch.Tensor, w_dkv_kr: torch.Tensor, cache: LatentCache,

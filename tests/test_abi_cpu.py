@@ -241,3 +241,31 @@ def test_status_codes_match_header():
         assert getattr(V, name) == value
     for name, value in (("VMLA_PATH_LATENT", 0), ("VMLA_PATH_DENSE", 1), ("VMLA_PATH_LATENT_FUSED", 2)):
         assert re.search(r"\b%s\s*=\s*%d\b" % (name, value), text), name
+
+
+def test_cache_checkpoint_round_trip(tmp_path):
+    """save / load restore the ring planes bit for bit (NaN-poisoned rows included) and frames_written;
+    a checkpoint of another configuration or kind is refused."""
+    import torch
+    cfg = TINY
+    cache = V.LatentCache(cfg, 2, device="cpu", fill=float("nan"))
+    g = torch.Generator().manual_seed(3)
+    cache.c[:, :20] = torch.randn((2, 20, cfg.d_c), generator=g)
+    cache.k_r[:, :20] = torch.randn((2, 20, cfg.d_rope), generator=g)
+    cache.struct.frames_written = 7
+    path = tmp_path / "layer0.pt"
+    cache.save(path)
+    back = V.LatentCache.load(path, cfg, device="cpu")
+    assert back.frames_written == 7 and back.batch == 2
+    assert torch.equal(back.c.view(torch.int32), cache.c.view(torch.int32))
+    assert torch.equal(back.k_r.view(torch.int32), cache.k_r.view(torch.int32))
+    assert back.struct.c == back.c.data_ptr()
+    with pytest.raises(ValueError, match="configuration"):
+        V.LatentCache.load(path, cfg.replace(window_frames=4), device="cpu")
+    with pytest.raises(ValueError, match="latent cache"):
+        V.DenseCache.load(path, cfg, device="cpu")
+    dense = V.DenseCache(cfg, 1, device="cpu", fill=0.5)
+    dense.struct.frames_written = 3
+    dense.save(tmp_path / "dense.pt")
+    dback = V.DenseCache.load(tmp_path / "dense.pt", cfg, device="cpu")
+    assert dback.frames_written == 3 and torch.equal(dback.k, dense.k) and torch.equal(dback.v, dense.v)
