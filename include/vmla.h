@@ -122,7 +122,10 @@ VMLA_API vmla_status vmla_compress_append_rows(const vmla_config* cfg, const voi
 /* Peer mappings of device buffers across processes (CUDA IPC).  vmla_ipc_export describes the buffer
  * holding dev_ptr (allocation handle + offset of dev_ptr in it); vmla_ipc_import maps it into this
  * process (another GPU's memory, reached over NVLink) and returns the matching pointer;
- * vmla_ipc_release unmaps it.  The exporter keeps its buffer alive until every importer released it. */
+ * vmla_ipc_release unmaps it.  The exporter keeps its buffer alive until every importer released it.
+ * The buffer must come from cudaMalloc (PyTorch's default caching allocator does); memory from the
+ * virtual-memory allocation API (PyTorch's expandable segments) cannot be exported this way and
+ * vmla_ipc_export returns VMLA_ERR_CUDA. */
 typedef struct {
   unsigned char bytes[64];
   int64_t offset;
