@@ -307,6 +307,13 @@ VMLA_API int32_t vmla_set_wait_timeout_ms(int32_t ms);
  * tile < 0 clears a pending request.  Nothing is faulted; later launches are unaffected. */
 VMLA_API void vmla_debug_drop_kv_tile(int32_t tile);
 
+/* Test hook of checked builds (built with VMLA_CHECKED=1, e.g. `build.py --checked`), whose kernels
+ * test every computed global store against its buffer's extent and, instead of storing outside it,
+ * record code 90 + site in the device status word: later launches record their buffers `bytes`
+ * shorter than they are, so that correct stores at the buffers' ends are reported (and skipped).
+ * 0 clears it.  Returns 1 in a checked build, 0 otherwise (where the hook has no effect). */
+VMLA_API int32_t vmla_debug_shrink_extents(int64_t bytes);
+
 /* Number of kernels the library has launched in this process (all entry points, all devices). */
 VMLA_API int64_t vmla_launch_count(void);
 

@@ -1,8 +1,11 @@
 """Build libvmla.so in-tree with nvcc for sm_100a.
 
-    python -m rank_latent_kv_vmla_b200.build [--force] [--jobs N]
+    python -m rank_latent_kv_vmla_b200.build [--force] [--jobs N] [--checked]
 
 Objects go to ``_build/`` at the repository root; the shared library is written next to this file.
+``--checked`` builds ``libvmla_checked.so`` (objects in ``_build_checked/``) with VMLA_CHECKED=1: every
+computed global store of the tensor-core kernels is tested against its buffer's extent (a store outside
+is skipped and reported in the device status word).  Select it with VMLA_LIBRARY=<path> at import.
 """
 from __future__ import annotations
 
@@ -20,6 +23,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libvmla.so")
+BUILD_CHECKED = os.path.join(ROOT, "_build_checked")
+LIB_CHECKED = os.path.join(PKG, "libvmla_checked.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden", "--expt-relaxed-constexpr",
@@ -52,13 +57,15 @@ def _compile(src: str, obj: str, extra):
     return r.stderr
 
 
-def build(force: bool = False, jobs: int = 0, extra=(), verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, jobs: int = 0, extra=(), verbose: bool = False, checked: bool = False) -> str:
+    build_dir, lib = (BUILD_CHECKED, LIB_CHECKED) if checked else (BUILD, LIB)
+    extra = list(extra) + (["-DVMLA_CHECKED=1"] if checked else [])
+    os.makedirs(build_dir, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = _headers()
     objs, todo = [], []
     for src in sources:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src] + headers + [__file__]):
             todo.append((src, obj))
@@ -68,14 +75,14 @@ def build(force: bool = False, jobs: int = 0, extra=(), verbose: bool = False) -
             for (src, _), log in zip(todo, ex.map(lambda so: _compile(so[0], so[1], extra), todo)):
                 if verbose and log:
                     print(f"--- {os.path.basename(src)}\n{log}", file=sys.stderr)
-    if force or todo or _stale(LIB, objs):
-        tmp = LIB + ".tmp"
+    if force or todo or _stale(lib, objs):
+        tmp = lib + ".tmp"
         cmd = [nvcc(), "-shared", "-o", tmp] + objs + ARCH
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 def main():
@@ -83,9 +90,11 @@ def main():
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--jobs", type=int, default=0)
     ap.add_argument("--ptxas-verbose", action="store_true", help="print register/smem use per kernel")
+    ap.add_argument("--checked", action="store_true", help="build libvmla_checked.so (bounds-checked stores)")
     a = ap.parse_args()
     extra = ["-Xptxas", "-v"] if a.ptxas_verbose else []
-    print(build(force=a.force or a.ptxas_verbose, jobs=a.jobs, extra=extra, verbose=a.ptxas_verbose))
+    print(build(force=a.force or a.ptxas_verbose, jobs=a.jobs, extra=extra, verbose=a.ptxas_verbose,
+                checked=a.checked))
 
 
 if __name__ == "__main__":

@@ -95,6 +95,7 @@ struct AttnParams {
   int d_nope;            // K of the absorbing MMA (multiple of 16, <= 128)
   int d_v;               // N of the value up-projection MMA (multiple of 32, <= BN)
   RopeTable rt;          // 3D-RoPE pairs of the query rotation
+  Span out_span, lse_span;   // extents of out and lse (checked builds)
 };
 
 // Compile-time plan of one kernel instance.
@@ -640,7 +641,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           for (int c = 0; c < p.d_v / 32; ++c) {
             tmem_ld32(tmem + lane_base + c * 32, o);
             tmem_ld_wait();
-            if (row_valid) {
+            if (row_valid && store_ok(p.out_span, out + orow * p.d_v + c * 32, 64, p.status, 9)) {
               uint4* dst = reinterpret_cast<uint4*>(out + orow * p.d_v + c * 32);
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
@@ -659,7 +660,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       for (int c = 0; c < (FUSED ? 0 : DV / 32); ++c) {
         tmem_ld32(tmem + lane_base + PL::kTmemO + c * 32, o);
         tmem_ld_wait();
-        if (row_valid) {
+        if (row_valid && store_ok(p.out_span, out + orow * DV + c * 32, 64, p.status, 7)) {
           uint4* dst = reinterpret_cast<uint4*>(out + orow * DV + c * 32);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -672,7 +673,8 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           }
         }
       }
-      if (row_valid && p.lse) p.lse[orow] = (m_ref + __log2f(l_row)) * 0.69314718055994530942f;
+      if (row_valid && p.lse && store_ok(p.lse_span, p.lse + orow, 4, p.status, 8))
+        p.lse[orow] = (m_ref + __log2f(l_row)) * 0.69314718055994530942f;
     }
   }
   tc_fence_before();
@@ -759,6 +761,8 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
   p.status = status;
   p.limit_ns = wait_limit_ns();
   p.drop_kv_tile = take_drop_kv_tile();
+  p.out_span = make_span(out, checked_extent((int64_t)batch * rows * cfg.d_c * 2));
+  p.lse_span = make_span(lse, checked_extent((int64_t)batch * rows * 4));
   const int n_tiles = batch * p.tiles_per_group;
   switch (cfg.d_c) {
     case 64: return launch_attention<1, 32, 1, true, kLatentBN, 2, true, false, false>(m, p, n_tiles, st);
@@ -844,6 +848,8 @@ cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t
   p.d_nope = dn;
   p.d_v = dv;
   p.rt = rt;
+  p.out_span = make_span(out, checked_extent((int64_t)batch * nq * H * dv * 2));
+  p.lse_span = make_span(lse, checked_extent((int64_t)batch * nq * H * 4));
   const int n_tiles = batch * H * p.tiles_per_group;
   switch (dc) {
     case 128: return launch_attention<2, 32, 2, true, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
@@ -885,6 +891,8 @@ cudaError_t tc_dense_mha(const vmla_config& cfg, int batch, int64_t nq, const vo
   p.status = status;
   p.limit_ns = wait_limit_ns();
   p.drop_kv_tile = -1;
+  p.out_span = make_span(out, checked_extent((int64_t)batch * nq * H * D * 2));
+  p.lse_span = make_span(lse, checked_extent((int64_t)batch * nq * H * 4));
   const int n_tiles = batch * H * p.tiles_per_group;
   return launch_attention<2, 0, 2, false, kBN, 2, true, false, false>(m, p, n_tiles, st);
 }

@@ -33,6 +33,15 @@ uint64_t wait_limit_ns() { return g_wait_limit_ns.load(); }
 
 int take_drop_kv_tile() { return g_drop_kv_tile.exchange(-1); }
 
+namespace {
+std::atomic<int64_t> g_shrink_extents{0};
+}
+
+int64_t checked_extent(int64_t bytes) {
+  const int64_t s = g_shrink_extents.load();
+  return bytes > s ? bytes - s : 0;
+}
+
 cudaError_t ensure_smem_attr(const void* kernel, int bytes, std::atomic<uint64_t>& done) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -78,3 +87,8 @@ extern "C" VMLA_API int32_t vmla_set_wait_timeout_ms(int32_t ms) {
 }
 
 extern "C" VMLA_API void vmla_debug_drop_kv_tile(int32_t tile) { vmla::g_drop_kv_tile.store(tile); }
+
+extern "C" VMLA_API int32_t vmla_debug_shrink_extents(int64_t bytes) {
+  vmla::g_shrink_extents.store(bytes > 0 ? bytes : 0);
+  return VMLA_CHECKED;
+}

@@ -15,6 +15,36 @@ struct TmaMaps5 {
   CUtensorMap wuk, wuv;   // fused latent attention: W^K_up and W^V_up
 };
 
+// Checked builds (compiled with -DVMLA_CHECKED=1): every computed global store of the tensor-core
+// kernels is tested against the extent of the buffer it writes; a store outside it is skipped and its
+// site (90 + site) is recorded in the device status word.  Release builds compile the test away.
+#ifndef VMLA_CHECKED
+#define VMLA_CHECKED 0
+#endif
+struct Span {
+  const void* base;
+  int64_t bytes;
+};
+__host__ __device__ inline Span make_span(const void* base, int64_t bytes) { return Span{base, bytes}; }
+#ifdef __CUDACC__
+__device__ __forceinline__ bool store_ok(const Span& s, const void* p, int bytes, int* status, int site) {
+#if VMLA_CHECKED
+  const char* b = static_cast<const char*>(s.base);
+  const char* q = static_cast<const char*>(p);
+  if (q < b || q + bytes > b + s.bytes) {
+    if (status) atomicCAS(status, 0, 90 + site);
+    return false;
+  }
+#else
+  (void)s; (void)p; (void)bytes; (void)status; (void)site;
+#endif
+  return true;
+}
+#endif
+// Extent of a buffer of `bytes` as the checked build records it: less `vmla_debug_shrink_extents`
+// bytes when that test hook is set, so that correct stores at the end of the buffer are reported.
+int64_t checked_extent(int64_t bytes);
+
 // Encode a 4-D bf16 tensor map {d0 (contiguous), d1, d2, d3} with byte strides s1, s2, s3 of the
 // three outer dimensions and box {b0, b1, b2, 1}; swizzle_bytes is 128, 64, 32 or 0.  Out-of-range
 // rows read as zeros.

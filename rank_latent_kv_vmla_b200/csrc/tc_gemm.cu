@@ -128,16 +128,23 @@ struct EpiCompress {
   static constexpr bool kRope = true;
   bf16* c[kMaxCacheDst]; bf16* k_r[kMaxCacheDst]; int n_dst;
   int d_c, d_rope; int64_t ntok, tok0, cap; FrameGeom g; RopeLookup rope;
+  Span c_span[kMaxCacheDst], kr_span[kMaxCacheDst]; int* status;
   __device__ void operator()(const float2* tab, int, int64_t m, int col0, float* v) const {
     const int64_t b = m / ntok, tok = tok0 + m % ntok;
     const int64_t row = b * cap + ring_row(g, tok);
     if (col0 < d_c) {
-      for (int d = 0; d < n_dst; ++d) store32(c[d] + row * d_c + col0, v);
+      for (int d = 0; d < n_dst; ++d) {
+        bf16* q = c[d] + row * d_c + col0;
+        if (store_ok(c_span[d], q, 64, status, 1)) store32(q, v);
+      }
     } else {
       const int64_t f = g.first_frame + tok / g.tokens_per_frame;
       const int64_t r = tok % g.tokens_per_frame;
       rope.rotate32(tab, (col0 - d_c) / 2, f, r / g.grid_w, r % g.grid_w, v);
-      for (int d = 0; d < n_dst; ++d) store32(k_r[d] + row * d_rope + (col0 - d_c), v);
+      for (int d = 0; d < n_dst; ++d) {
+        bf16* q = k_r[d] + row * d_rope + (col0 - d_c);
+        if (store_ok(kr_span[d], q, 64, status, 2)) store32(q, v);
+      }
     }
     // stores to other GPUs' memory: make them visible system-wide before this thread goes on
     if (n_dst > 1) __threadfence_system();
@@ -148,8 +155,10 @@ struct EpiCompress {
 struct EpiAbsorb {
   static constexpr bool kRope = true;
   bf16* q_abs; const bf16* q_rope; int heads, d_c, d_rope; int64_t nq; FrameGeom g; RopeLookup rope;
+  Span span; int* status;
   __device__ void operator()(const float2* tab, int h, int64_t m, int col0, float* v) const {
-    store32(q_abs + (m * heads + h) * (d_c + d_rope) + col0, v);
+    bf16* q = q_abs + (m * heads + h) * (d_c + d_rope) + col0;
+    if (store_ok(span, q, 64, status, 3)) store32(q, v);
   }
   // RoPE3D(q^rope) of row m, head h -> q_abs[m, h, d_c : d_c + d_rope]
   __device__ void finish(const float2* tab, int h, int64_t m) const {
@@ -168,7 +177,8 @@ struct EpiAbsorb {
         for (int t = 0; t < 8; ++t) v[8 * q + t] = __bfloat162float(e[t]);
       }
       rope.rotate32(tab, c0 / 2, f, r / g.grid_w, r % g.grid_w, v);
-      store32(q_abs + (m * heads + h) * (d_c + d_rope) + d_c + c0, v);
+      bf16* q = q_abs + (m * heads + h) * (d_c + d_rope) + d_c + c0;
+      if (store_ok(span, q, 64, status, 3)) store32(q, v);
     }
   }
 };
@@ -177,8 +187,10 @@ struct EpiValueUp {
   static constexpr bool kRope = false;
   RopeLookup rope;   // unused
   bf16* out; int heads, d_v;
+  Span span; int* status;
   __device__ void operator()(const float2* tab, int h, int64_t m, int col0, float* v) const {
-    store32(out + (m * heads + h) * d_v + col0, v);
+    bf16* q = out + (m * heads + h) * d_v + col0;
+    if (store_ok(span, q, 64, status, 4)) store32(q, v);
   }
   __device__ void finish(const float2*, int, int64_t) const {}
 };
@@ -186,6 +198,7 @@ struct EpiValueUp {
 struct EpiDense {
   static constexpr bool kRope = true;
   bf16* k; bf16* v; int heads, d_nope, d_h, d_v; int64_t ntok, cap; FrameGeom g; RopeLookup rope;
+  Span k_span, v_span; int* status;
   __device__ void operator()(const float2* tab, int, int64_t m, int col0, float* x) const {
     const int64_t b = m / ntok, tok = m % ntok;
     const int64_t row = b * cap + ring_row(g, tok);
@@ -196,10 +209,12 @@ struct EpiDense {
         const int64_t r = tok % g.tokens_per_frame;
         rope.rotate32(tab, (cc - d_nope) / 2, f, r / g.grid_w, r % g.grid_w, x);
       }
-      store32(k + (row * heads + hh) * d_h + cc, x);
+      bf16* q = k + (row * heads + hh) * d_h + cc;
+      if (store_ok(k_span, q, 64, status, 5)) store32(q, x);
     } else {
       const int cv = col0 - heads * d_h;
-      store32(v + (row * heads + cv / d_v) * d_v + cv % d_v, x);
+      bf16* q = v + (row * heads + cv / d_v) * d_v + cv % d_v;
+      if (store_ok(v_span, q, 64, status, 6)) store32(q, x);
     }
   }
   __device__ void finish(const float2*, int, int64_t) const {}
@@ -517,10 +532,14 @@ cudaError_t tc_compress_rows(const vmla_config& cfg, int batch, int64_t tok0, in
     return e;
   GemmShape sh{M, N, K, 0, wait_limit_ns(), device_status_ptr()};
   EpiCompress epi{};
+  const int64_t cap_rows = (int64_t)batch * cfg.window_frames * cfg.grid_h * cfg.grid_w;
   for (int d = 0; d < n_dst; ++d) {
     epi.c[d] = (bf16*)dst[d].c;
     epi.k_r[d] = (bf16*)dst[d].k_r;
+    epi.c_span[d] = make_span(dst[d].c, checked_extent(cap_rows * cfg.d_c * 2));
+    epi.kr_span[d] = make_span(dst[d].k_r, checked_extent(cap_rows * cfg.d_rope * 2));
   }
+  epi.status = device_status_ptr();
   epi.n_dst = n_dst;
   epi.d_c = cfg.d_c;
   epi.d_rope = cfg.d_rope;
@@ -547,6 +566,8 @@ cudaError_t tc_absorb_q(const vmla_config& cfg, int batch, int64_t nq, const voi
   GemmShape sh{M, N, K, 1, wait_limit_ns(), device_status_ptr()};
   EpiAbsorb epi{(bf16*)q_abs, (const bf16*)q_rope, H, cfg.d_c, cfg.d_rope, nq, g,
                 make_rope_lookup(rt, g, (int)(nq / ((int64_t)cfg.grid_h * cfg.grid_w)))};
+  epi.span = make_span(q_abs, checked_extent(M * H * (cfg.d_c + cfg.d_rope) * 2));
+  epi.status = device_status_ptr();
   return dispatch_bn<true>(N, ma, mb, sh, H, epi, st);
 }
 
@@ -563,6 +584,8 @@ cudaError_t tc_value_up(const vmla_config& cfg, int batch, int64_t n_tokens, con
     return e;
   GemmShape sh{M, N, K, 1, wait_limit_ns(), device_status_ptr()};
   EpiValueUp epi{RopeLookup{}, (bf16*)out, H, N};
+  epi.span = make_span(out, checked_extent(M * H * N * 2));
+  epi.status = device_status_ptr();
   return dispatch_bn<false>(N, ma, mb, sh, H, epi, st);
 }
 
@@ -583,6 +606,10 @@ cudaError_t tc_dense_append(const vmla_config& cfg, int batch, const void* x, co
   GemmShape sh{M, N, K, 0, wait_limit_ns(), device_status_ptr()};
   EpiDense epi{(bf16*)k, (bf16*)v, cfg.n_heads, cfg.d_nope, d_h, cfg.d_v, ntok,
                (int64_t)cfg.window_frames * cfg.grid_h * cfg.grid_w, g, make_rope_lookup(rt, g, cfg.chunk_frames)};
+  const int64_t dense_rows = (int64_t)batch * cfg.window_frames * cfg.grid_h * cfg.grid_w * cfg.n_heads;
+  epi.k_span = make_span(k, checked_extent(dense_rows * d_h * 2));
+  epi.v_span = make_span(v, checked_extent(dense_rows * cfg.d_v * 2));
+  epi.status = device_status_ptr();
   return dispatch_bn<false>(bn, ma, mb, sh, 1, epi, st);
 }
 

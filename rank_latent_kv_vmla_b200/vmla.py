@@ -14,7 +14,8 @@ import torch
 
 from .config import VMLA_BF16, VMLA_F32, VmlaConfig
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvmla.so")
+# VMLA_LIBRARY selects another build of the library (e.g. the bounds-checked libvmla_checked.so)
+_LIB_PATH = os.environ.get("VMLA_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvmla.so")
 
 VMLA_OK, VMLA_ERR_INVALID_ARG, VMLA_ERR_UNSUPPORTED, VMLA_ERR_MISALIGNED, VMLA_ERR_CUDA, \
     VMLA_ERR_TIMEOUT = range(6)
@@ -28,7 +29,7 @@ EXPORTED = ("vmla_compress_append", "vmla_absorb_q", "vmla_latent_attention", "v
             "vmla_latent_attention_fused", "vmla_executor_workspace_bytes", "vmla_executor_create",
             "vmla_executor_submit", "vmla_executor_wait", "vmla_executor_destroy",
             "vmla_compress_append_rows", "vmla_latent_attention_fused_rows", "vmla_ipc_export",
-            "vmla_ipc_import", "vmla_ipc_release")
+            "vmla_ipc_import", "vmla_ipc_release", "vmla_debug_shrink_extents")
 
 
 class VmlaError(RuntimeError):
@@ -113,6 +114,8 @@ def _load():
     lib.vmla_last_error_detail.restype = ctypes.c_char_p
     lib.vmla_debug_drop_kv_tile.argtypes = [I32]
     lib.vmla_debug_drop_kv_tile.restype = None
+    lib.vmla_debug_shrink_extents.argtypes = [I64]
+    lib.vmla_debug_shrink_extents.restype = I32
     lib.vmla_set_wait_timeout_ms.argtypes = [I32]
     lib.vmla_set_wait_timeout_ms.restype = I32
     lib.vmla_abi_version.argtypes = []
