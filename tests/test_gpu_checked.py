@@ -30,7 +30,7 @@ w_kv = synthetic.draw_dense_weights(cfg, 4).to(dev)
 lc = V.LatentCache(cfg, B, device=dev)
 dc = V.DenseCache(cfg, B, device=dev)
 reps = [V.LatentCache(cfg, B, device=dev) for _ in range(3)]
-shards = token_shards(cfg.chunk_tokens, 3)
+shards = token_shards(cfg.chunk_tokens, 3, align=8)        # 120 tokens: 40 + 40 + 40
 def status(what):
     code = V.device_status()
     print(what, code)

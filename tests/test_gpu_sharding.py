@@ -38,7 +38,10 @@ def test_virtual_ranks_one_gpu(V, world):
     orc = OracleLayer(cfg, inp, B)
     reps = [V.LatentCache(cfg, B, device=DEV, fill=float("nan")) for _ in range(world)]
     ref = V.LatentCache(cfg, B, device=DEV, fill=float("nan"))
-    shards = token_shards(cfg.chunk_tokens, world)
+    # 120 tokens per chunk: shards split at multiples of 8 (40 + 40 + 40, or 64 + 56), so every virtual
+    # rank holds rows and the ranges start inside 128-token tiles
+    shards = token_shards(cfg.chunk_tokens, world, align=8)
+    assert all(cnt > 0 for _, cnt in shards)
     for k in range(n_chunks):
         x, qn, qr = (_to(t) for t in synthetic.draw_chunk(cfg, B, 950 + 10 * world + k))
         f0 = ref.frames_written
