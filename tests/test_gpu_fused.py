@@ -1,7 +1,8 @@
 """GPU parity of the fused call (absorbed query + latent attention + value up-projection in one
 kernel): against the float64 oracle on every streamed chunk, and against the three-call path on the
-same inputs.  Tiles are 128 tokens of one head, so the mid config's 480 tokens give a ragged last
-tile per head; the Wan-shaped layer is checked at full size on sampled tokens."""
+same inputs.  Tiles are 128 tokens of one head: the mid config's 120-token chunks are one ragged tile
+per head, a 12 x 12 grid gives 288-token chunks (2.25 tiles per head), and the Wan-shaped layer (37
+tiles per head) is checked at full size on sampled tokens."""
 import numpy as np
 import pytest
 import torch
@@ -64,6 +65,12 @@ def _stream_fused(V, cfg, batch, n_steps, seed, rows=None):
 def test_mid_fused_streaming(V):
     """4 two-frame chunks into a 5-frame window (partial, full, wrapping), B = 2, every call."""
     _stream_fused(V, MID, batch=2, n_steps=4, seed=3030)
+
+
+def test_mid_fused_streaming_multitile(V):
+    """288-token chunks (12 x 12 grid, F = 2): two full tiles and a ragged third per head, 4 chunks into a
+    5-frame window (the ring wraps), B = 2."""
+    _stream_fused(V, MID.replace(grid_h=12, grid_w=12), batch=2, n_steps=4, seed=3050)
 
 
 @pytest.mark.parametrize("d_c", [128, 256])
