@@ -1,7 +1,9 @@
 // Projection GEMMs of the VideoMLA path on the sm_100a tensor cores (tcgen05 + TMEM + TMA), each
 // with its own fused epilogue:
 //   compress_append  [c ; W^KR x] = [W^KV_down ; W^KR] x, 3D-RoPE on the last d_rope columns, bf16
-//                    store into the ring rows of the chunk's frames (Method items 1 and 3);
+//                    store into the ring rows of the chunk's frames (Method items 1 and 3); also a
+//                    token range of the chunk into several replicas of the ring (peer mappings), and
+//                    the column tile narrows to 128 / 64 when the row tiles alone leave SMs idle;
 //   absorb_q         q~_h = (W^K_up,h)^T q^nope_h per head (B operand read MN-major from W^K_up as
 //                    stored), plus RoPE3D(q^rope_h) written beside it (Method items 2 and 3);
 //   value_up         o_h = W^V_up,h o~_h per head (Method item 2);
@@ -11,7 +13,8 @@
 // k-tiles with TMA into a shared-memory ring, warp 1 owns TMEM and issues tcgen05.mma (K = 16 per
 // instruction, fp32 accumulation) into one of two TMEM accumulators, and warps 2-5 read the other
 // accumulator back (one thread per row) and run the epilogue, so a tile's epilogue overlaps the next
-// tile's loads and MMAs.
+// tile's loads and MMAs.  The epilogue warps also build the CTA's 3D-RoPE cos/sin table while the
+// first loads and MMAs run.  In checked builds every epilogue store is tested against its buffer.
 #include <cuda.h>
 
 #include <atomic>
