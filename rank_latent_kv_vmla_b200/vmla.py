@@ -1,8 +1,13 @@
 """Python binding of libvmla (ctypes).  Argument marshalling only: every step runs in the library's
 CUDA kernels; PyTorch supplies device memory and the current CUDA stream.
 
-Importing this module loads ``libvmla.so`` from the package directory and raises if it is missing:
-there is no fallback implementation.
+Importing this module loads ``libvmla.so`` from the package directory (or the library named by the
+VMLA_LIBRARY environment variable, e.g. the bounds-checked ``libvmla_checked.so``) and raises if it is
+missing: there is no fallback implementation.
+
+Besides the per-call functions the module offers LatentCache / DenseCache (ring planes with
+checkpoint save / load), Executor (layer steps with host buffers, copies overlapped with the
+kernels), plan_capacity, and the row-range and IPC calls used by ``sharding``.
 """
 from __future__ import annotations
 
