@@ -53,3 +53,20 @@ def test_executor_matches_synchronous_path(V):
         assert torch.equal(ex_caches[l].c, ref_caches[l].c)
         assert torch.equal(ex_caches[l].k_r, ref_caches[l].k_r)
     assert V.device_status() == 0
+
+
+def test_executor_rejects_bad_submissions(V):
+    cfg = MID
+    w, wuk, wuv = (t.to(DEV) for t in synthetic.draw_weights(cfg, 72))
+    x, qn, qr = (t.pin_memory() for t in synthetic.draw_chunk(cfg, 2, 73))
+    ho = torch.empty((2, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16).pin_memory()
+    with V.Executor(cfg, 2) as ex:
+        with pytest.raises(V.VmlaError):
+            ex.submit(V.LatentCache(cfg, 1, device=DEV), w, wuk, wuv, x, qn, qr, ho)     # batch 1 cache
+        with pytest.raises(ValueError):
+            ex.submit(V.LatentCache(cfg, 2, device=DEV), w, wuk, wuv, x.cuda(), qn, qr, ho)   # device input
+        cache = V.LatentCache(cfg, 2, device=DEV)
+        ex.submit(cache, w, wuk, wuv, x, qn, qr, ho)          # the executor still works afterwards
+        ex.wait()
+        assert cache.frames_written == cfg.chunk_frames
+    assert V.device_status() == 0
