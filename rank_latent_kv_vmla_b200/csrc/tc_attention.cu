@@ -1,9 +1,9 @@
-// Flash-style attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA) for
-//  * the VideoMLA latent cache (absorbed form): one KV "head" shared by every query head, keys
-//    [c ; k^R] (d_c + 32 wide) and values c (d_c wide) read from the same shared-memory stage
-//    (VideoMLA technical summary, Method items 2-3: per-head keys and values are reconstructed from
-//    the shared latent; here the reconstruction is folded into the query and applied after the sum);
-//  * the dense per-head comparison layer (d_h = d_v = 128 per head).
+// Flash-style attention on the sm_100a tensor cores (tcgen05 + TMEM + TMA) over the VideoMLA latent
+// cache (absorbed form): one KV "head" shared by every query head, keys [c ; k^R] (d_c + 32 wide) and
+// values c (d_c wide) read from the same shared-memory stage (VideoMLA technical summary, Method items
+// 2-3: per-head keys and values are reconstructed from the shared latent; here the reconstruction is
+// folded into the query and applied after the sum).  The dense per-head comparison layer has its own
+// kernel (tc_dense.cu).
 //
 // One CTA owns one tile of 128 query rows and streams every visible KV tile of BN keys:
 //   warp 4      TMA producer: KV tiles into an NST-deep shared-memory ring (and the Q tile when Q
@@ -18,7 +18,7 @@
 //               latency-bound with one warp per SM sub-partition, so it uses 3-input max and packed
 //               f32x2 FMA / add instructions.
 // Q lives in TMEM (S = Q K^T then reads only K from shared memory) where the TMEM budget allows it
-// with 128-key tiles: d_c = 64 / 128 and the dense layer.  For d_c = 192 / 256 (2 S buffers + O leave
+// with 128-key tiles: d_c = 64 / 128.  For d_c = 192 / 256 (2 S buffers + O leave
 // no room for Q at 128 keys) Q stays in shared memory; a Q-in-TMEM build with 96-key tiles was
 // measured slower.  The KV ring is released by tcgen05.commit after the P V MMAs that last read a stage.
 //
@@ -76,12 +76,11 @@ __device__ __forceinline__ void rope_rotate_mufu(const RopeTable& rt, int p, int
 
 struct AttnParams {
   const void* q;         // query rows (used when Q is kept in TMEM)
-  int rows_per_b;        // query rows per batch element (latent: Nq*H, dense: Nq)
+  int rows_per_b;        // query rows per batch element (token-major: Nq*H, head-major: Nq)
   int tiles_per_group;   // query tiles per (batch[, head]) group
-  int heads;             // dense: heads per token (tile groups are (b, h)); latent: n = row / heads
-  int dense;             // 1 for the per-head dense layer
+  int heads;             // head-major: tile groups are (b, h); token-major: token = row / heads
   int64_t nq;            // query tokens per batch element
-  int head_major;        // tiles are 128 tokens of one head (dense and fused layers)
+  int head_major;        // tiles are 128 tokens of one head (the fused layer)
   int64_t tok0;          // head-major: query row r is token tok0 + r of the call (a token range)
   FrameGeom g;
   float scale_log2;      // softmax_scale * log2(e)
@@ -99,14 +98,14 @@ struct AttnParams {
 };
 
 // Compile-time plan of one kernel instance.
-//   KB    64-column boxes of the key tile from the first key plane (c, or dense K)
+//   KB    64-column boxes of the key tile from the c plane
 //   KR    width of the rope box (0 or 32, 64-byte swizzle)
-//   VB    64-column boxes of the value tile (V = the first VB key boxes when V_ALIAS)
+//   VB    64-column boxes of the value tile: V = the first VB key boxes (the latent c)
 //   BN    keys per KV tile;  NS  TMEM S buffers (the MMA runs NS - 1 tiles ahead of P V)
 //   Q_TMEM  whether Q lives in TMEM (the A operand of S = Q K^T) or in shared memory
 //   ONES  V is extended by 16 columns of ones in shared memory, so that the P V MMA also produces
 //         the row sum of P in O's column DV (the softmax then needs no add chains)
-template <int KB, int KR, int VB, bool V_ALIAS, int BN, int NS, bool Q_TMEM, bool ONES, bool FUSED>
+template <int KB, int KR, int VB, int BN, int NS, bool Q_TMEM, bool ONES, bool FUSED>
 struct Plan {
   static constexpr int kDQK = 64 * KB + KR;
   static constexpr int kDV = 64 * VB;
@@ -114,13 +113,12 @@ struct Plan {
   static constexpr int kBox = BN * 128;                 // [BN x 64] bf16 box, 128-byte swizzle
   static constexpr int kRopeBox = BN * 64;              // [BN x 32] bf16 box, 64-byte swizzle
   static constexpr int kQBytes = Q_TMEM ? 0 : (KB * kBlockM * 128 + (KR ? kBlockM * 64 : 0));
-  // stage layout: K boxes | V boxes (unless aliased) | ones box | rope box
-  static constexpr int kVOff = V_ALIAS ? 0 : KB * kBox;
-  static constexpr int kOnesOff = kVOff + VB * kBox;
-  static constexpr int kRopeOff = (V_ALIAS && !ONES) ? KB * kBox : kOnesOff + (ONES ? kBox : 0);
+  // stage layout: c boxes (K, and V = the first VB of them) | ones box | rope box
+  static constexpr int kOnesOff = KB * kBox;
+  static constexpr int kRopeOff = kOnesOff + (ONES ? kBox : 0);
   static constexpr int kStageRaw = kRopeOff + (KR ? kRopeBox : 0);
   static constexpr int kStageBytes = (kStageRaw + 1023) / 1024 * 1024;
-  static constexpr int kLoadBytes = KB * kBox + (V_ALIAS ? 0 : VB * kBox) + (KR ? kRopeBox : 0);
+  static constexpr int kLoadBytes = KB * kBox + (KR ? kRopeBox : 0);
   static constexpr int kAuxBytes = 512;                 // barriers
   static constexpr int kBudget = 232448 - 1024 - kAuxBytes;
   static constexpr int kFit = (kBudget - kQBytes) / kStageBytes;
@@ -136,18 +134,18 @@ struct Plan {
   static_assert(!ONES || Q_TMEM, "the ones box is filled by the warps that also write Q into TMEM");
   static_assert(kNPV <= 256 && kNPV % 16 == 0, "P V MMA shape");
   // fused: q^nope (two 64-column boxes) and then O / l must fit the Q buffer
-  static_assert(!FUSED || (!Q_TMEM && V_ALIAS && KR == 32 && !ONES && KB >= 2 &&
+  static_assert(!FUSED || (!Q_TMEM && KR == 32 && !ONES && KB >= 2 &&
                            kQBytes >= 2 * kBlockM * 128 && kQBytes >= VB * kBlockM * 128),
                 "fused layout");
 };
 
-template <int KB, int KR, int VB, bool V_ALIAS, int BN, int NS, bool Q_TMEM, bool ONES, bool FUSED>
+template <int KB, int KR, int VB, int BN, int NS, bool Q_TMEM, bool ONES, bool FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
 attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_qr,
                  const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_kr,
-                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_wuk,
+                 const __grid_constant__ CUtensorMap map_wuk,
                  const __grid_constant__ CUtensorMap map_wuv, const AttnParams p) {
-  using PL = Plan<KB, KR, VB, V_ALIAS, BN, NS, Q_TMEM, ONES, FUSED>;
+  using PL = Plan<KB, KR, VB, BN, NS, Q_TMEM, ONES, FUSED>;
   constexpr int NST = PL::kStages;
   constexpr int DV = PL::kDV;
   constexpr int DQK = PL::kDQK;
@@ -178,7 +176,6 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   const int row0 = (tile % p.tiles_per_group) * kBlockM;      // first query row of the tile
   const int b = p.head_major ? group / p.heads : group;
   const int h = p.head_major ? group % p.heads : 0;
-  const int kv_h = p.dense ? h : 0;                            // head coordinate of the KV maps
   const int tok_div = p.head_major ? 1 : p.heads;              // query row -> token
   const int last_row = min(row0 + kBlockM, p.rows_per_b) - 1;
   const int64_t tok_base = p.head_major ? p.tok0 : 0;
@@ -217,7 +214,6 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     // ================= TMA producer =================
     if (elect_one()) {
       tma_prefetch_desc(&map_k);
-      if (!V_ALIAS) tma_prefetch_desc(&map_v);
       if (!Q_TMEM && !FUSED) {
         mbar_arrive_expect_tx(bar_q, PL::kQBytes);
         for (int i = 0; i < KB; ++i) tma_load_4d(sQ + i * kBlockM * 128, &map_q, bar_q, 64 * i, h, row0, b);
@@ -251,11 +247,8 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         uint8_t* stage = sKV + st * PL::kStageBytes;
         mbar_arrive_expect_tx(kv_full + st, PL::kLoadBytes);
         const int krow = j * BN;
-        for (int i = 0; i < KB; ++i) tma_load_4d(stage + i * PL::kBox, &map_k, kv_full + st, 64 * i, kv_h, krow, b);
+        for (int i = 0; i < KB; ++i) tma_load_4d(stage + i * PL::kBox, &map_k, kv_full + st, 64 * i, 0, krow, b);
         if (KR) tma_load_4d(stage + PL::kRopeOff, &map_kr, kv_full + st, 0, 0, krow, b);
-        if (!V_ALIAS)
-          for (int i = 0; i < VB; ++i)
-            tma_load_4d(stage + PL::kVOff + i * PL::kBox, &map_v, kv_full + st, 64 * i, kv_h, krow, b);
       }
       if (FUSED && issued == n_kv && claim(n_kv)) {
         // W^V_up,h (d_c/64 K-major boxes of [d_v rows][64 columns]) as load n_kv of the ring
@@ -302,7 +295,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       // still produce the second half's P
       auto issue_pv = [&](int jp) -> bool {
         const int bp = jp % NS;
-        const uint32_t v_base = kv_base + (jp % NST) * PL::kStageBytes + PL::kVOff;
+        const uint32_t v_base = kv_base + (jp % NST) * PL::kStageBytes;
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k) {
           if (k == 0 || k == BN / 32) {
@@ -685,14 +678,14 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   }
 }
 
-template <int KB, int KR, int VB, bool V_ALIAS, int BN, int NS, bool Q_TMEM, bool ONES, bool FUSED>
-cudaError_t launch_attention(const TmaMaps5& m, const AttnParams& p, int n_tiles, cudaStream_t st) {
-  using PL = Plan<KB, KR, VB, V_ALIAS, BN, NS, Q_TMEM, ONES, FUSED>;
-  auto kern = attention_kernel<KB, KR, VB, V_ALIAS, BN, NS, Q_TMEM, ONES, FUSED>;
+template <int KB, int KR, int VB, int BN, int NS, bool Q_TMEM, bool ONES, bool FUSED>
+cudaError_t launch_attention(const AttnMaps& m, const AttnParams& p, int n_tiles, cudaStream_t st) {
+  using PL = Plan<KB, KR, VB, BN, NS, Q_TMEM, ONES, FUSED>;
+  auto kern = attention_kernel<KB, KR, VB, BN, NS, Q_TMEM, ONES, FUSED>;
   static std::atomic<uint64_t> done{0};
   cudaError_t attr_err = ensure_smem_attr((const void*)kern, PL::kSmemBytes, done);
   if (attr_err != cudaSuccess) return attr_err;
-  kern<<<n_tiles, kThreads, PL::kSmemBytes, st>>>(m.q, m.qr, m.k, m.kr, m.v, m.wuk, m.wuv, p);
+  kern<<<n_tiles, kThreads, PL::kSmemBytes, st>>>(m.q, m.qr, m.k, m.kr, m.wuk, m.wuv, p);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -700,7 +693,7 @@ cudaError_t launch_attention(const TmaMaps5& m, const AttnParams& p, int n_tiles
 // Instances (measured on B200; the softmax warps bound these kernels, the MMA side alone reaches the
 // full tensor rate in every one of them):
 //   latent d_c = 192 / 256: Q in shared memory, 128-key tiles, two S buffers (fastest per key);
-//   latent d_c = 64 / 128 and the dense layer: Q in TMEM, 128-key tiles, two S buffers.
+//   latent d_c = 64 / 128: Q in TMEM, 128-key tiles, two S buffers.
 // The three-buffer / 64-key / ones-column variant of the template is correct but slower at these
 // shapes (its per-tile fixed costs outweigh the shorter dependency chain).
 constexpr int kLatentBN = 128;
@@ -716,15 +709,6 @@ vmla_status tc_check_latent_attention(const vmla_config& c) {
   return VMLA_OK;
 }
 
-vmla_status tc_check_dense_mha(const vmla_config& c) {
-  const int d_h = c.d_nope + c.d_rope;
-  if (d_h != 128 || c.d_v != 128) {
-    set_tc_reason("tensor-core dense attention needs d_h == d_v == 128");
-    return VMLA_ERR_UNSUPPORTED;
-  }
-  return VMLA_OK;
-}
-
 cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, const void* q_abs,
                                 const void* c, const void* k_r, int64_t cap, int64_t valid_rows,
                                 const FrameGeom& g, float scale, void* out, float* lse, int* status,
@@ -732,7 +716,7 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
   const int H = cfg.n_heads, dqk = cfg.d_c + cfg.d_rope;
   const int64_t rows = nq * H;
   const int kv_box_rows = kLatentBN;
-  TmaMaps5 m{};
+  AttnMaps m{};
   cudaError_t e;
   // q_abs [B, Nq*H, d_qk] viewed as 4D {d_qk, 1, Nq*H, B} (only read by TMA when Q stays in smem)
   if ((e = make_map_4d(&m.q, q_abs, dqk, 1, rows, batch, (int64_t)dqk * 2, (int64_t)dqk * 2,
@@ -743,7 +727,6 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
                        cap * cfg.d_c * 2, 64, 1, kv_box_rows, 128)) != cudaSuccess) return e;
   if ((e = make_map_4d(&m.kr, k_r, 32, 1, valid_rows, batch, 64, 64, cap * 64, 32, 1, kv_box_rows, 64)) != cudaSuccess)
     return e;
-  m.v = m.k;
   m.wuk = m.k;
   m.wuv = m.k;
   AttnParams p{};
@@ -751,7 +734,6 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
   p.rows_per_b = (int)rows;
   p.tiles_per_group = (int)((rows + kBlockM - 1) / kBlockM);
   p.heads = H;
-  p.dense = 0;
   p.head_major = 0;
   p.nq = nq;
   p.g = g;
@@ -765,10 +747,10 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
   p.lse_span = make_span(lse, checked_extent((int64_t)batch * rows * 4));
   const int n_tiles = batch * p.tiles_per_group;
   switch (cfg.d_c) {
-    case 64: return launch_attention<1, 32, 1, true, kLatentBN, 2, true, false, false>(m, p, n_tiles, st);
-    case 128: return launch_attention<2, 32, 2, true, kLatentBN, 2, true, false, false>(m, p, n_tiles, st);
-    case 192: return launch_attention<3, 32, 3, true, kLatentBN, 2, false, false, false>(m, p, n_tiles, st);
-    default: return launch_attention<4, 32, 4, true, kLatentBN, 2, false, false, false>(m, p, n_tiles, st);
+    case 64: return launch_attention<1, 32, 1, kLatentBN, 2, true, false, false>(m, p, n_tiles, st);
+    case 128: return launch_attention<2, 32, 2, kLatentBN, 2, true, false, false>(m, p, n_tiles, st);
+    case 192: return launch_attention<3, 32, 3, kLatentBN, 2, false, false, false>(m, p, n_tiles, st);
+    default: return launch_attention<4, 32, 4, kLatentBN, 2, false, false, false>(m, p, n_tiles, st);
   }
 }
 
@@ -776,7 +758,7 @@ namespace {
 
 // Fused instances: Q in shared memory (the prologue writes it there), 128-key tiles, two S buffers.
 template <int KB>
-using FusedPlan = Plan<KB, 32, KB, true, kLatentBN, 2, false, false, true>;
+using FusedPlan = Plan<KB, 32, KB, kLatentBN, 2, false, false, true>;
 
 template <int KB>
 bool fused_fits(int d_nope, int d_v) {
@@ -811,7 +793,7 @@ cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t
                                       const FrameGeom& g, const RopeTable& rt, float scale, void* out, float* lse,
                                       int* status, cudaStream_t st) {
   const int H = cfg.n_heads, dn = cfg.d_nope, dc = cfg.d_c, dv = cfg.d_v;
-  TmaMaps5 m{};
+  AttnMaps m{};
   cudaError_t e;
   // q^nope [B, Nq, H, d_nope] as {d_nope, H, Nq, B}: a 128-token box of one head
   if ((e = make_map_4d(&m.q, q_nope, dn, H, nq, batch, (int64_t)dn * 2, (int64_t)H * dn * 2,
@@ -821,7 +803,6 @@ cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t
                        cap * dc * 2, 64, 1, kLatentBN, 128)) != cudaSuccess) return e;
   if ((e = make_map_4d(&m.kr, k_r, 32, 1, valid_rows, batch, 64, 64, cap * 64, 32, 1, kLatentBN, 64)) != cudaSuccess)
     return e;
-  m.v = m.k;
   // W^K_up [H, d_nope, d_c] as {d_c, d_nope, H, 1}: [d_nope rows][64 columns] boxes (MN-major B)
   if ((e = make_map_4d(&m.wuk, w_uk, dc, dn, H, 1, (int64_t)dc * 2, (int64_t)dn * dc * 2,
                        (int64_t)H * dn * dc * 2, 64, dn, 1, 128)) != cudaSuccess) return e;
@@ -833,7 +814,6 @@ cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t
   p.rows_per_b = (int)nq;
   p.tiles_per_group = (int)((nq + kBlockM - 1) / kBlockM);
   p.heads = H;
-  p.dense = 0;
   p.head_major = 1;
   p.tok0 = tok0;
   p.nq = nq;
@@ -852,49 +832,10 @@ cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t
   p.lse_span = make_span(lse, checked_extent((int64_t)batch * nq * H * 4));
   const int n_tiles = batch * H * p.tiles_per_group;
   switch (dc) {
-    case 128: return launch_attention<2, 32, 2, true, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
-    case 192: return launch_attention<3, 32, 3, true, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
-    default: return launch_attention<4, 32, 4, true, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
+    case 128: return launch_attention<2, 32, 2, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
+    case 192: return launch_attention<3, 32, 3, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
+    default: return launch_attention<4, 32, 4, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
   }
-}
-
-cudaError_t tc_dense_mha(const vmla_config& cfg, int batch, int64_t nq, const void* q, const void* k,
-                         const void* v, int64_t cap, int64_t valid_rows, const FrameGeom& g,
-                         float scale, void* out, float* lse, int* status, cudaStream_t st) {
-  const int H = cfg.n_heads;
-  const int D = 128;
-  constexpr int kBN = 128;
-  TmaMaps5 m{};
-  cudaError_t e;
-  if ((e = make_map_4d(&m.q, q, D, H, nq, batch, D * 2, (int64_t)H * D * 2, nq * H * D * 2, 64, 1, kBlockM,
-                       128)) != cudaSuccess) return e;
-  m.qr = m.q;
-  if ((e = make_map_4d(&m.k, k, D, H, valid_rows, batch, D * 2, (int64_t)H * D * 2, cap * H * D * 2, 64, 1,
-                       kBN, 128)) != cudaSuccess) return e;
-  m.kr = m.k;
-  if ((e = make_map_4d(&m.v, v, D, H, valid_rows, batch, D * 2, (int64_t)H * D * 2, cap * H * D * 2, 64, 1,
-                       kBN, 128)) != cudaSuccess) return e;
-  m.wuk = m.k;
-  m.wuv = m.k;
-  AttnParams p{};
-  p.q = q;
-  p.rows_per_b = (int)nq;
-  p.tiles_per_group = (int)((nq + kBlockM - 1) / kBlockM);
-  p.heads = H;
-  p.dense = 1;
-  p.head_major = 1;
-  p.nq = nq;
-  p.g = g;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.out = out;
-  p.lse = lse;
-  p.status = status;
-  p.limit_ns = wait_limit_ns();
-  p.drop_kv_tile = -1;
-  p.out_span = make_span(out, checked_extent((int64_t)batch * nq * H * D * 2));
-  p.lse_span = make_span(lse, checked_extent((int64_t)batch * nq * H * 4));
-  const int n_tiles = batch * H * p.tiles_per_group;
-  return launch_attention<2, 0, 2, false, kBN, 2, true, false, false>(m, p, n_tiles, st);
 }
 
 }  // namespace vmla

@@ -10,9 +10,11 @@
 
 namespace vmla {
 
-struct TmaMaps5 {
-  CUtensorMap q, qr, k, kr, v;
-  CUtensorMap wuk, wuv;   // fused latent attention: W^K_up and W^V_up
+// Tensor maps of one latent attention launch: query boxes (q, and its rope part qr), the cache planes
+// (k = c, also read as V; kr = k^R) and, for the fused layer, W^K_up and W^V_up.
+struct AttnMaps {
+  CUtensorMap q, qr, k, kr;
+  CUtensorMap wuk, wuv;
 };
 
 // Checked builds (compiled with -DVMLA_CHECKED=1): every computed global store of the tensor-core
