@@ -13,8 +13,8 @@
 //   warps 0-3   one thread per query row (= TMEM lane): first the Q row into TMEM (when Q is kept
 //               in TMEM), then per tile the softmax: masked running max with a lazy rescale of O (only
 //               when the max grows by more than 2^8), exp2 (a quarter of them by an FMA-pipe
-//               polynomial), row sum, P to TMEM in two key halves, each released to the P V MMAs by
-//               its own barrier; finally O / l to global memory and the log-sum-exp.  The softmax is
+//               polynomial), row sum, P to TMEM in four parts of 32 keys, each released to the P V
+//               MMAs by its own barrier; finally O / l to global memory and the log-sum-exp.  The softmax is
 //               latency-bound with one warp per SM sub-partition, so it uses 3-input max and packed
 //               f32x2 FMA / add instructions.
 // Q lives in TMEM (S = Q K^T then reads only K from shared memory) where the TMEM budget allows it
@@ -55,6 +55,12 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #define VMLA_EXP2_POLY_PAIRS 2
 #endif
 constexpr int kPolyPairs = VMLA_EXP2_POLY_PAIRS;
+// P of a tile is released to the P V MMAs in this many parts (consecutive key ranges), so that the
+// MMAs of the first parts run while the softmax warps still exponentiate the rest.
+#ifndef VMLA_P_PARTS
+#define VMLA_P_PARTS 4
+#endif
+constexpr int kPParts = VMLA_P_PARTS;
 
 // Rotation of query pair p for the fused prologue: the angle is formed and reduced to [-pi, pi] in
 // double precision (large frame indices lose nothing), then the MUFU sine / cosine (absolute error
@@ -148,6 +154,8 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   using PL = Plan<KB, KR, VB, BN, NS, Q_TMEM, ONES, FUSED>;
   constexpr int NST = PL::kStages;
   constexpr int DV = PL::kDV;
+  constexpr int kStepsPerPart = BN / 16 / kPParts;     // 16-key MMA steps per released part of P
+  static_assert((BN / 16) % kPParts == 0, "P parts");
   constexpr int DQK = PL::kDQK;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -158,8 +166,8 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   uint64_t* kv_full = bars + 1;           // NST
   uint64_t* kv_empty = kv_full + NST;     // NST
   uint64_t* s_full = kv_empty + NST;      // NS
-  uint64_t* p_ready = s_full + NS;        // [NS][2]: P of the first / second half of the tile's keys
-  uint64_t* pv_done = p_ready + 2 * NS;   // NS: P V of a tile of that S buffer completed
+  uint64_t* p_ready = s_full + NS;        // [NS][kPParts]: P of one part of the tile's keys written
+  uint64_t* pv_done = p_ready + kPParts * NS;  // NS: P V of a tile of that S buffer completed
   uint64_t* drain = pv_done + NS;         // 1
   uint64_t* bar_pro = drain + 1;          // fused: q^nope and W^K_up,h landed
   uint64_t* qa_full = bar_pro + 1;        // fused: q~ = q^nope W^K_up,h complete in TMEM
@@ -188,8 +196,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     for (int s = 0; s < NST; ++s) { mbar_init(kv_full + s, 1); mbar_init(kv_empty + s, 1); }
     for (int s = 0; s < NS; ++s) {
       mbar_init(s_full + s, 1);
-      mbar_init(p_ready + 2 * s, 128);
-      mbar_init(p_ready + 2 * s + 1, 128);
+      for (int q = 0; q < kPParts; ++q) mbar_init(p_ready + kPParts * s + q, 128);
       mbar_init(pv_done + s, 1);
     }
     mbar_init(drain, 1);
@@ -291,15 +298,16 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         }
       }
       ok = ok && mbar_wait(bar_q, 0, abort_flag, p.status, 2, p.limit_ns);
-      // P V of tile jp in two halves of the keys: the first half's MMAs run while the softmax warps
-      // still produce the second half's P
+      // P V of tile jp in kPParts parts of the keys: the first parts' MMAs run while the softmax warps
+      // still produce the rest of P
       auto issue_pv = [&](int jp) -> bool {
         const int bp = jp % NS;
         const uint32_t v_base = kv_base + (jp % NST) * PL::kStageBytes;
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k) {
-          if (k == 0 || k == BN / 32) {
-            if (!mbar_wait(p_ready + 2 * bp + (k ? 1 : 0), (jp / NS) & 1, abort_flag, p.status, 3, p.limit_ns))
+          if (k % kStepsPerPart == 0) {
+            if (!mbar_wait(p_ready + kPParts * bp + k / kStepsPerPart, (jp / NS) & 1, abort_flag, p.status, 3,
+                           p.limit_ns))
               return false;
             tc_fence_after();
           }
@@ -576,10 +584,10 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st8(tmem + lane_base + bj * BN + c * 8, pk);
-        if (c == BN / 32 - 1) {                       // first half of the keys: release it to P V
+        if ((c + 1) % kStepsPerPart == 0 && c + 1 < BN / 16) {   // a part of the keys: release it to P V
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(p_ready + 2 * bj);
+          mbar_arrive(p_ready + kPParts * bj + c / kStepsPerPart);
         }
       }
       if (!ONES) {
@@ -590,7 +598,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_ready + 2 * bj + 1);
+      mbar_arrive(p_ready + kPParts * bj + kPParts - 1);
     }
     bool fin = ok && mbar_wait(drain, 0, abort_flag, p.status, 7, p.limit_ns);
     fin = __all_sync(0xffffffffu, fin && !*abort_flag);

@@ -8,7 +8,7 @@
 // no per-tile exchange between the warpgroups); the two partial results are merged once, at the end.
 // The exponentials of a tile still share each sub-partition's MUFU and FMA pipes (~1000 of the ~1330
 // cycles a half takes, measured), and the tile period is the chain S_j -> softmax -> P_j V_j ->
-// S_{j+2} spread over the two S buffers.
+// S_{j+2} spread over the two S buffers; releasing P in 32-key parts shortens its tail.
 //
 // One CTA owns one tile of 128 query rows of one (batch, head) and streams every visible KV tile:
 //   warp 8      TMA producer: the Q tile once, then K and V tiles of 128 keys into a 3-deep ring;
@@ -18,7 +18,7 @@
 //   warps 0-3   keys 0-63 of every tile, warps 4-7 keys 64-127; one thread per query row (= TMEM lane,
 //               warps w and w + 4 share the lanes): masked running max with a lazy rescale of O_w (only
 //               when the max grows by more than 2^8), exp2 (3/8 by an FMA-pipe polynomial), row
-//               sum, P released to the MMA warp by the half's own barrier.  Finally the halves swap
+//               sum, P released to the MMA warp in two parts of 32 keys.  Finally the halves swap
 //               (max, sum) through shared memory and each warpgroup writes 64 of the 128 output
 //               columns of o = (O_0 2^(m_0 - m) + O_1 2^(m_1 - m)) / l, warps 0-3 also the log-sum-exp.
 // TMEM: S buffers at columns [0, 128) and [128, 256), O_0 at [256, 384), O_1 at [384, 512).
@@ -58,6 +58,13 @@ constexpr float kRescaleThreshold = 8.0f;     // log2 units
 #define VMLA_DENSE_EXP2_POLY_PAIRS 3
 #endif
 constexpr int kPolyPairs = VMLA_DENSE_EXP2_POLY_PAIRS;
+// Each key half releases its P to the P V MMAs in this many parts.
+#ifndef VMLA_DENSE_P_PARTS
+#define VMLA_DENSE_P_PARTS 2
+#endif
+constexpr int kPParts = VMLA_DENSE_P_PARTS;
+constexpr int kStepsPerPart = kHalf / 16 / kPParts;   // 16-key MMA steps per released part
+static_assert((kHalf / 16) % kPParts == 0, "P parts");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kTmemO + 2 * kHead <= kTmemCols, "TMEM budget");
 
@@ -87,8 +94,8 @@ dense_attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
   uint64_t* kv_full = bars + 1;              // [kStages]
   uint64_t* kv_empty = kv_full + kStages;    // [kStages]
   uint64_t* s_full = kv_empty + kStages;     // [2 S buffers]
-  uint64_t* p_ready = s_full + 2;            // [2 S buffers][2 key halves], 128 arrivals each
-  uint64_t* pv_done = p_ready + 4;           // [2 S buffers][2 key halves]: that half's P V completed
+  uint64_t* p_ready = s_full + 2;            // [2 S buffers][2 key halves][kPParts], 128 arrivals each
+  uint64_t* pv_done = p_ready + 4 * kPParts; // [2 S buffers][2 key halves]: that half's P V completed
   uint64_t* drain = pv_done + 4;             // every MMA of the CTA completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -108,7 +115,8 @@ dense_attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
     mbar_init(bar_q, 1);
     for (int s = 0; s < kStages; ++s) { mbar_init(kv_full + s, 1); mbar_init(kv_empty + s, 1); }
     for (int s = 0; s < 2; ++s) mbar_init(s_full + s, 1);
-    for (int i = 0; i < 4; ++i) { mbar_init(p_ready + i, 128); mbar_init(pv_done + i, 1); }
+    for (int i = 0; i < 4 * kPParts; ++i) mbar_init(p_ready + i, 128);
+    for (int i = 0; i < 4; ++i) mbar_init(pv_done + i, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -163,10 +171,14 @@ dense_attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
         const int bp = jp & 1;
         const uint32_t v_base = kv_base + (jp % kStages) * kStageBytes + 2 * kBox;
         for (int w = 0; w < 2; ++w) {
-          if (!mbar_wait(p_ready + 2 * bp + w, (jp >> 1) & 1, abort_flag, p.status, 23, p.limit_ns)) return false;
-          tc_fence_after();
 #pragma unroll
           for (int k = 0; k < kHalf / 16; ++k) {
+            if (k % kStepsPerPart == 0) {
+              if (!mbar_wait(p_ready + (2 * bp + w) * kPParts + k / kStepsPerPart, (jp >> 1) & 1, abort_flag,
+                             p.status, 23, p.limit_ns))
+                return false;
+              tc_fence_after();
+            }
             // V tile [128 keys][128 columns] as MN-major operand: 8-key groups 1024 B apart (SBO), the two
             // 64-column boxes kBox apart (LBO); 16 keys are 2048 B.  P of keys 64w + 16k .. + 15 sits in
             // the 8 columns at 64w + 8k of the S buffer.
@@ -291,6 +303,11 @@ dense_attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st8(s_addr + c * 8, pk);
+        if ((c + 1) % kStepsPerPart == 0 && c + 1 < kHalf / 16) {   // a part of the half: release it
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(p_ready + (2 * bj + wg) * kPParts + c / kStepsPerPart);
+        }
       }
       fadd2(ls[0], ls[1], ls[4], ls[5]);
       fadd2(ls[2], ls[3], ls[6], ls[7]);
@@ -298,7 +315,7 @@ dense_attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
       l_sum += ls[0] + ls[1];
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_ready + 2 * bj + wg);
+      mbar_arrive(p_ready + (2 * bj + wg) * kPParts + kPParts - 1);
     }
     bool fin = ok && mbar_wait(drain, 0, abort_flag, p.status, 27, p.limit_ns);
     fin = __all_sync(0xffffffffu, fin && !*abort_flag);
