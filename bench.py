@@ -408,8 +408,8 @@ def _capacity_workload(V, synthetic, dev, clocks, budget=60 * 10**9, n_layers=30
     for name, cfg, dense in (("latent_dc64", WAN.replace(d_c=64), False),
                              ("latent_dc128", WAN.replace(d_c=128), False),
                              ("latent_dc192", WAN, False), ("dense", WAN, True)):
-        # the latent step runs fused where the fused kernel supports the shape (d_c >= 128)
-        fused = (not dense) and cfg.d_c >= 128
+        # the latent step runs fused where the fused kernel supports the shape (d_c >= 128 here)
+        fused = (not dense) and V.fused_supported(cfg)
         plan = V.plan_capacity(cfg, n_layers, budget, dense=dense, fused=fused)
         row = {"path": name + ("_fused" if fused else ""), **plan}
         if name in ("latent_dc192", "dense"):
@@ -479,7 +479,7 @@ def run_workload(args):
                    "query_tokens_per_s": B * cfg.chunk_tokens / (ms * 1e-3),
                    "cache_bytes_per_layer": V.latent_cache_bytes(cfg, B),
                    "cache_fraction_of_dense": V.latent_cache_bytes(cfg, B) / V.dense_cache_bytes(cfg, B)}
-            if d_c >= 128:
+            if V.fused_supported(cfg):
                 # the fused call: absorb + attention + value-up in one launch (what the layer step runs)
                 wuv = inp.w_uv.to(dev)
                 o_f = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)

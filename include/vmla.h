@@ -233,6 +233,11 @@ VMLA_API vmla_status vmla_dense_mha(const vmla_config* cfg, const void* q, const
 VMLA_API vmla_status vmla_check_attention_window(const vmla_config* cfg, int64_t frames_written,
                                                  int64_t first_frame, int32_t n_query_chunks);
 
+/* Host-only check whether vmla_latent_attention_fused supports this configuration: VMLA_OK, or
+ * VMLA_ERR_UNSUPPORTED with the reason in the detail text (VMLA_ERR_INVALID_ARG for an invalid cfg).
+ * Launches nothing; callers use it to choose between the fused call and the three separate calls. */
+VMLA_API vmla_status vmla_check_fused(const vmla_config* cfg);
+
 /* Synchronise `stream`, then read and clear the device status word of the current device:
  * *code = 0 if no device-side wait ran out since the last call, else a nonzero code naming the wait.
  * Returns VMLA_ERR_TIMEOUT when *code != 0. */

@@ -603,6 +603,16 @@ vmla_status vmla_check_attention_window(const vmla_config* cfg, int64_t frames_w
   return check_window(*cfg, frames_written, first_frame, n_query_chunks);
 }
 
+vmla_status vmla_check_fused(const vmla_config* cfg) {
+  vmla_status s = check_config(cfg);
+  if (s != VMLA_OK) return s;
+  if (cfg->dtype != VMLA_BF16)
+    return fail(VMLA_ERR_UNSUPPORTED, "the fused call runs on the bf16 tensor-core path only");
+  s = tc_check_fused_attention(*cfg);
+  if (s != VMLA_OK) return fail(s, "%s", tc_last_reason());
+  return VMLA_OK;
+}
+
 vmla_status vmla_device_status(void* stream, int32_t* code) {
   if (!code) return fail(VMLA_ERR_INVALID_ARG, "code is NULL");
   cudaError_t e = cudaStreamSynchronize(as_stream(stream));

@@ -27,7 +27,8 @@ VMLA_OK, VMLA_ERR_INVALID_ARG, VMLA_ERR_UNSUPPORTED, VMLA_ERR_MISALIGNED, VMLA_E
 
 EXPORTED = ("vmla_compress_append", "vmla_absorb_q", "vmla_latent_attention", "vmla_value_up",
             "vmla_rope_q", "vmla_dense_append", "vmla_dense_mha", "vmla_device_status",
-            "vmla_check_attention_window", "vmla_set_wait_timeout_ms", "vmla_debug_drop_kv_tile",
+            "vmla_check_attention_window", "vmla_check_fused", "vmla_set_wait_timeout_ms",
+            "vmla_debug_drop_kv_tile",
             "vmla_latent_cache_bytes", "vmla_dense_cache_bytes", "vmla_launch_count",
             "vmla_status_string", "vmla_last_error_detail", "vmla_abi_version",
             "vmla_compress_rewrite", "vmla_dense_rewrite", "vmla_plan_capacity",
@@ -88,6 +89,7 @@ def _load():
         "vmla_dense_mha": [cfgp, VP, P(CDenseCache), I64, I32, VP, VP, VP],
         "vmla_device_status": [VP, P(I32)],
         "vmla_check_attention_window": [cfgp, I64, I64, I32],
+        "vmla_check_fused": [cfgp],
         "vmla_compress_rewrite": [cfgp, VP, VP, P(CCache), VP],
         "vmla_dense_rewrite": [cfgp, VP, VP, P(CDenseCache), VP],
         "vmla_plan_capacity": [cfgp, I32, I32, I64, I64, I64, P(CCapacity)],
@@ -420,6 +422,16 @@ def check_attention_window(cfg: VmlaConfig, frames_written: int, first_frame: in
     check(LIB.vmla_check_attention_window(ctypes.byref(cc), frames_written, first_frame, n_query_chunks))
 
 
+def fused_supported(cfg: VmlaConfig) -> bool:
+    """Whether latent_attention_fused supports this configuration (host-only library check)."""
+    cc = c_config(cfg)
+    st = LIB.vmla_check_fused(ctypes.byref(cc))
+    if st == VMLA_ERR_UNSUPPORTED:
+        return False
+    check(st)
+    return True
+
+
 def set_wait_timeout_ms(ms: int) -> int:
     """Bound (ms) of every device-side wait of later launches; returns the previous bound."""
     return int(LIB.vmla_set_wait_timeout_ms(int(ms)))
@@ -585,8 +597,7 @@ def layer_step(cfg: VmlaConfig, x: torch.Tensor, q_nope: torch.Tensor, q_rope: t
     (default: for bf16 configs whose shapes it supports) or the three separate calls."""
     bufs = bufs if bufs is not None else {}
     if fused is None:
-        fused = cfg.dtype == VMLA_BF16 and cfg.d_rope == 32 and cfg.d_c in (128, 192, 256) and \
-            cfg.d_nope % 16 == 0 and 16 <= cfg.d_nope <= 128 and cfg.d_v % 32 == 0 and 32 <= cfg.d_v <= 128
+        fused = fused_supported(cfg)
     f0 = cache.frames_written
     compress_append(cfg, x, w_dkv_kr, cache, f0)
     if fused:
@@ -601,5 +612,5 @@ __all__ = ["LIB", "VmlaError", "LatentCache", "DenseCache", "compress_append", "
            "launch_count", "latent_cache_bytes", "dense_cache_bytes", "layer_step", "c_config",
            "compress_rewrite", "dense_rewrite", "plan_capacity", "CCapacity", "latent_attention_fused", "Executor",
            "compress_append_rows", "latent_attention_fused_rows", "ipc_export", "ipc_import", "ipc_release",
-           "CIpcHandle",
+           "CIpcHandle", "check_attention_window", "fused_supported",
            "CConfig", "CCache", "CDenseCache", "EXPORTED", "VMLA_F32", "VMLA_BF16"]

@@ -269,3 +269,25 @@ def test_cache_checkpoint_round_trip(tmp_path):
     dense.save(tmp_path / "dense.pt")
     dback = V.DenseCache.load(tmp_path / "dense.pt", cfg, device="cpu")
     assert dback.frames_written == 3 and torch.equal(dback.k, dense.k) and torch.equal(dback.v, dense.v)
+
+
+@pytest.mark.parametrize("cfg,ok", [
+    (WAN, True),
+    (WAN.replace(d_c=128), True),
+    (WAN.replace(d_c=256), True),
+    (WAN.replace(d_c=64), False),        # the fused kernel needs d_c in {128, 192, 256}
+    (WAN.replace(d_nope=104, rope_pairs_t=6), False),   # d_nope not a multiple of 16
+    (TINY, False),                       # fp32 runs on the SIMT path only
+])
+def test_fused_support_query(cfg, ok):
+    """vmla_check_fused is host-only and agrees with what vmla_latent_attention_fused accepts."""
+    cc = V.c_config(cfg)
+    st, d = _status(V.LIB.vmla_check_fused, ctypes.byref(cc))
+    assert (st == V.VMLA_OK) == ok, d
+    assert V.fused_supported(cfg) == ok
+    if not ok:
+        assert st == V.VMLA_ERR_UNSUPPORTED and d
+        cache = _cache(frames_written=cfg.window_frames)
+        st2, _ = _status(V.LIB.vmla_latent_attention_fused, ctypes.byref(cc), FAKE, FAKE, FAKE, FAKE,
+                         ctypes.byref(cache), cfg.window_frames - cfg.chunk_frames, 1, FAKE, None, None)
+        assert st2 == V.VMLA_ERR_UNSUPPORTED
