@@ -305,9 +305,9 @@ VMLA_API vmla_status vmla_executor_destroy(vmla_executor* ex);   /* waits for pe
  * kernel stop, record a nonzero code for vmla_device_status() and return. */
 VMLA_API int32_t vmla_set_wait_timeout_ms(int32_t ms);
 
-/* Test hook for the bounded-wait path: the next bf16 latent attention launch (vmla_latent_attention or
- * one of the fused calls) does not load KV tile `tile` (keys tile*128 .. tile*128+127) of any query
- * tile, so the wait for it runs out, the kernel winds down without writing its outputs and
+/* Test hook for the bounded-wait path: the next bf16 attention launch (vmla_latent_attention, one of
+ * the fused calls or vmla_dense_mha) does not load KV tile `tile` (keys tile*128 .. tile*128+127) of
+ * any query tile, so the wait for it runs out, the kernel winds down without writing its outputs and
  * vmla_device_status() reports a nonzero code.
  * tile < 0 clears a pending request.  Nothing is faulted; later launches are unaffected. */
 VMLA_API void vmla_debug_drop_kv_tile(int32_t tile);

@@ -79,6 +79,7 @@ struct DenseParams {
   float* lse;            // [B, Nq, H] or null
   int* status;
   uint64_t limit_ns;
+  int drop_kv_tile;      // test hook: this KV tile is never loaded (-1: none)
   Span out_span, lse_span;
 };
 
@@ -145,6 +146,7 @@ dense_attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
         if (j >= kStages && !mbar_wait(kv_empty + st, ((j / kStages) - 1) & 1, abort_flag, p.status, 21, p.limit_ns))
           break;
         issued = j + 1;
+        if (j == p.drop_kv_tile) continue;
         uint8_t* stage = sKV + st * kStageBytes;
         mbar_arrive_expect_tx(kv_full + st, kStageBytes);
         const int krow = j * kBN;
@@ -155,7 +157,7 @@ dense_attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_c
         // let the copies already issued land before the CTA exits
         mbar_wait(bar_q, 0, &zero_flag, nullptr, 0, p.limit_ns);
         for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
-          mbar_wait(kv_full + j % kStages, (j / kStages) & 1, &zero_flag, nullptr, 0, p.limit_ns);
+          if (j != p.drop_kv_tile) mbar_wait(kv_full + j % kStages, (j / kStages) & 1, &zero_flag, nullptr, 0, p.limit_ns);
       }
     }
   } else if (warp == 9) {
@@ -412,6 +414,7 @@ cudaError_t tc_dense_mha(const vmla_config& cfg, int batch, int64_t nq, const vo
   p.lse = lse;
   p.status = status;
   p.limit_ns = wait_limit_ns();
+  p.drop_kv_tile = take_drop_kv_tile();
   p.out_span = make_span(out, checked_extent((int64_t)batch * nq * H * D * 2));
   p.lse_span = make_span(lse, checked_extent((int64_t)batch * nq * H * 4));
   const int n_tiles = batch * H * p.tiles_per_group;

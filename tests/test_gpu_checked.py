@@ -80,9 +80,9 @@ print("CODES", code_c, code_a)
 def test_checked_build_finds_no_store_outside_its_buffer():
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    if not os.path.exists(LIB):
-        from rank_latent_kv_vmla_b200 import build
-        build.build(checked=True)
+    # incremental: recompiles only what changed since the in-tree checked library was built
+    from rank_latent_kv_vmla_b200 import build
+    build.build(checked=True)
     env = dict(os.environ, VMLA_LIBRARY=LIB)
     r = subprocess.run([sys.executable, "-c", "ROOT = %r\n" % ROOT + SCRIPT], env=env, capture_output=True,
                        text=True, timeout=600)

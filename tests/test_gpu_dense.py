@@ -109,3 +109,36 @@ def test_batch_of_eight_runs_are_bit_identical(V):
     assert torch.equal(o1, o2)
     for b in range(8):
         assert_close(f64(o1[b]), orc.reference(b, inp.q_nope, inp.q_rope, f0)["o"], cfg, f"dense o b{b}")
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(V):
+    """A KV tile the dense kernel never loads: the MMA warp's wait for it runs out, both softmax halves
+    and the producer wind down (the producer does not wait for the missing copy), vmla_device_status
+    reports the code, and the next call on the same context is correct."""
+    cfg = MID
+    inp = synthetic.draw_layer(cfg, batch=1, seed=76, n_chunks=3)
+    orc = OracleLayer(cfg, inp, 1)
+    w_kv = _to(round_to(cfg, dense_weights_from_latent(inp, cfg)))
+    cache = V.DenseCache(cfg, 1, device=DEV)
+    for x in inp.x_chunks:
+        f0 = cache.frames_written
+        V.dense_append(cfg, _to(x), w_kv, cache)
+        orc.append(x)
+    q = V.rope_q(cfg, _to(inp.q_nope), _to(inp.q_rope), f0)
+    torch.cuda.synchronize()
+    assert V.device_status() == 0
+    old = V.set_wait_timeout_ms(20)
+    try:
+        V.debug_drop_kv_tile(1)
+        V.dense_mha(cfg, q, cache, f0)
+        torch.cuda.synchronize()
+        assert V.device_status() != 0
+        assert V.device_status() == 0          # reading clears it
+    finally:
+        V.debug_drop_kv_tile(-1)
+        V.set_wait_timeout_ms(old)
+    o = V.dense_mha(cfg, q, cache, f0)
+    torch.cuda.synchronize()
+    assert V.device_status() == 0
+    assert_close(f64(o[0]), orc.reference(0, inp.q_nope, inp.q_rope, f0)["o"], cfg, "dense o after a timed-out launch")
+
