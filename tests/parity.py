@@ -139,3 +139,14 @@ def dense_weights_from_latent(inp: synthetic.LayerInputs, cfg: VmlaConfig) -> np
     keys = [np.concatenate([w_uk[h] @ w_dkv, w_kr]) for h in range(cfg.n_heads)]
     vals = [w_uv[h] @ w_dkv for h in range(cfg.n_heads)]
     return np.concatenate(keys + vals)
+
+
+def sample_rows(cfg, nq_tokens, n=64):
+    """Query tokens to check: first and last tiles, frame and chunk boundaries, and a spread."""
+    T = cfg.tokens_per_frame
+    picks = {0, 1, 2, 10, 11, nq_tokens - 1, nq_tokens - 2, nq_tokens - 11}
+    for f in range(1, nq_tokens // T):
+        picks.update({f * T - 1, f * T})
+    spread = np.linspace(0, nq_tokens - 1, n - len(picks), dtype=np.int64)
+    picks.update(int(s) for s in spread)
+    return np.array(sorted(p for p in picks if 0 <= p < nq_tokens))[:max(n, len(picks))]

@@ -3,14 +3,16 @@
   * one-token frames: 1-3 visible keys, so the second half of the only tile is fully masked;
   * a window of many tiles with a ragged last tile (the second half of the last tile masked);
   * the whole window as one block-causal multi-chunk query set (rows of one tile see different ends);
-  * a batch of several sequences.
+  * a batch of several sequences;
+  * the Wan-1.3B shapes at full size (256 KV tiles, a ragged 37th query tile per head), sampled rows.
 The dense weights are W_K,h = [W^K_up,h W^KV_down ; W^KR] and W_V,h = W^V_up,h W^KV_down, so the
 float64 oracle's latent layer is the reference for o and the log-sum-exp."""
 import pytest
 import torch
 
 import synthetic
-from parity import MID, OracleLayer, assert_close, dense_weights_from_latent, f64, round_to
+from parity import MID, OracleLayer, assert_close, dense_weights_from_latent, f64, round_to, sample_rows
+from rank_latent_kv_vmla_b200.config import WAN
 
 pytestmark = pytest.mark.gpu
 
@@ -141,4 +143,27 @@ def test_bounded_wait_reports_timeout_and_context_survives(V):
     torch.cuda.synchronize()
     assert V.device_status() == 0
     assert_close(f64(o[0]), orc.reference(0, inp.q_nope, inp.q_rope, f0)["o"], cfg, "dense o after a timed-out launch")
+
+
+def test_wan_full_size_sampled(V):
+    """The dense layer at the Wan-1.3B shapes the bench times: 8 chunks streamed into the 21-frame
+    window (the last evicts frames 0-2), then the newest chunk's queries over all 32760 keys; o and the
+    log-sum-exp on sampled rows (first and last tiles, frame boundaries, a spread) of every head."""
+    cfg = WAN
+    inp = synthetic.draw_layer(cfg, batch=1, seed=1236, n_chunks=8)
+    orc = OracleLayer(cfg, inp, 1)
+    w_kv = _to(round_to(cfg, dense_weights_from_latent(inp, cfg)))
+    cache = V.DenseCache(cfg, 1, device=DEV, fill=float("nan"))
+    for x in inp.x_chunks:
+        f0 = cache.frames_written
+        V.dense_append(cfg, _to(x), w_kv, cache)
+        orc.append(x)
+    q = V.rope_q(cfg, _to(inp.q_nope), _to(inp.q_rope), f0)
+    o, lse = V.dense_mha(cfg, q, cache, f0, want_lse=True)
+    torch.cuda.synchronize()
+    assert V.device_status() == 0
+    rows = sample_rows(cfg, cfg.chunk_tokens)
+    ref = orc.reference(0, inp.q_nope, inp.q_rope, f0, rows=rows)
+    assert_close(f64(o[0][rows]), ref["o"], cfg, "dense o")
+    assert_close(f64(lse[0][rows]), ref["lse"], cfg, "dense lse")
 

@@ -10,7 +10,7 @@ import torch
 from oracle import vmla_oracle as O
 from rank_latent_kv_vmla_b200.config import TINY, WAN, VMLA_BF16
 import synthetic
-from parity import (MID, OracleLayer, assert_close, dense_weights_from_latent, f64, round_to,
+from parity import (MID, OracleLayer, assert_close, dense_weights_from_latent, f64, round_to, sample_rows,
                     pairs)
 
 pytestmark = pytest.mark.gpu
@@ -231,17 +231,6 @@ def test_tiny_fp32_dense_path(V):
     assert_close(f64(o_d[0]), ref["o"], cfg, "dense o")
 
 
-def _sample_rows(cfg, nq_tokens, n=64):
-    """Query tokens to check: first and last tiles, frame and chunk boundaries, and a spread."""
-    T = cfg.tokens_per_frame
-    picks = {0, 1, 2, 10, 11, nq_tokens - 1, nq_tokens - 2, nq_tokens - 11}
-    for f in range(1, nq_tokens // T):
-        picks.update({f * T - 1, f * T})
-    spread = np.linspace(0, nq_tokens - 1, n - len(picks), dtype=np.int64)
-    picks.update(int(s) for s in spread)
-    return np.array(sorted(p for p in picks if 0 <= p < nq_tokens))[:max(n, len(picks))]
-
-
 @pytest.mark.parametrize("batch", [1, 2])
 def test_wan_full_size_sampled(V, batch):
     """The Wan-1.3B-shaped layer at full size: 8 chunks streamed into the 21-frame window (the last
@@ -262,7 +251,7 @@ def test_wan_full_size_sampled(V, batch):
     o = V.value_up(cfg, o_lat, _to(inp.w_uv))
     torch.cuda.synchronize()
     assert V.device_status() == 0
-    rows = _sample_rows(cfg, cfg.chunk_tokens)
+    rows = sample_rows(cfg, cfg.chunk_tokens)
     q_ref = orc.q_abs(inp.q_nope, inp.q_rope, f0)
     for b in sorted({0, batch - 1}):
         c_ref, kr_ref, written = orc.ring(b)
