@@ -291,3 +291,60 @@ def test_fused_support_query(cfg, ok):
         st2, _ = _status(V.LIB.vmla_latent_attention_fused, ctypes.byref(cc), FAKE, FAKE, FAKE, FAKE,
                          ctypes.byref(cache), cfg.window_frames - cfg.chunk_frames, 1, FAKE, None, None)
         assert st2 == V.VMLA_ERR_UNSUPPORTED
+
+
+_MIDLIKE = WAN.replace(grid_h=6, grid_w=10, chunk_frames=2, window_frames=5)   # 120-token chunks, bf16
+
+
+@pytest.mark.parametrize("begin,n", [
+    (0, 0),                 # empty range
+    (-8, 16),               # negative start
+    (64, 64),               # past the chunk's 120 tokens
+])
+def test_row_range_compress_rejects_bad_ranges(begin, n):
+    """vmla_compress_append_rows validates the token range, the replica list and every replica's
+    frames_written on the host, and launches nothing for a rejected call (FAKE device pointers are
+    never dereferenced)."""
+    cfg = _MIDLIKE
+    cc = V.c_config(cfg)
+    reps = (V.CCache * 2)(_cache(), _cache())
+    st, d = _status(V.LIB.vmla_compress_append_rows, ctypes.byref(cc), FAKE, FAKE, 0, begin, n, reps, 2, None)
+    assert st == V.VMLA_ERR_INVALID_ARG and "token range" in d, d
+
+
+def test_row_range_compress_rejects_bad_replicas():
+    cfg = _MIDLIKE
+    cc = V.c_config(cfg)
+    call = lambda reps, k, ff=0: _status(V.LIB.vmla_compress_append_rows, ctypes.byref(cc), FAKE, FAKE, ff, 0, 8,
+                                         reps, k, None)
+    reps = (V.CCache * 9)(*[_cache() for _ in range(9)])
+    assert call(reps, 0)[0] == V.VMLA_ERR_INVALID_ARG                 # no replica
+    assert call(reps, 9)[0] == V.VMLA_ERR_INVALID_ARG                 # more than the kernel's 8 destinations
+    assert call(None, 1)[0] == V.VMLA_ERR_INVALID_ARG
+    bad = (V.CCache * 2)(_cache(), _cache(c=None))
+    st, d = call(bad, 2)
+    assert st == V.VMLA_ERR_INVALID_ARG and "NULL" in d, d
+    bad = (V.CCache * 2)(_cache(), _cache(batch=2))
+    st, d = call(bad, 2)
+    assert st == V.VMLA_ERR_INVALID_ARG and "batch" in d, d
+    bad = (V.CCache * 2)(_cache(), _cache(frames_written=2))
+    st, d = call(bad, 2)
+    assert st == V.VMLA_ERR_INVALID_ARG and "frames_written" in d, d
+    bad = (V.CCache * 2)(_cache(), _cache(c=FAKE + 8))
+    assert call(bad, 2)[0] == V.VMLA_ERR_MISALIGNED
+    st, d = _status(V.LIB.vmla_compress_append_rows, ctypes.byref(V.c_config(TINY)), FAKE, FAKE, 0, 0, 8,
+                    (V.CCache * 1)(_cache()), 1, None)
+    assert st == V.VMLA_ERR_UNSUPPORTED                                # fp32 has no row-range path
+
+
+@pytest.mark.parametrize("begin,n", [(0, 0), (-1, 8), (100, 40), (0, 121)])
+def test_row_range_fused_rejects_bad_ranges(begin, n):
+    """vmla_latent_attention_fused_rows: the token range must lie inside the call's query tokens."""
+    cfg = _MIDLIKE
+    cc = V.c_config(cfg)
+    cache = _cache(frames_written=cfg.window_frames)
+    f0 = cfg.window_frames - cfg.chunk_frames
+    st, d = _status(V.LIB.vmla_latent_attention_fused_rows, ctypes.byref(cc), FAKE, FAKE, FAKE, FAKE,
+                    ctypes.byref(cache), f0, 1, begin, n, FAKE, None, None)
+    assert st == V.VMLA_ERR_INVALID_ARG and "token range" in d, d
+
