@@ -348,3 +348,21 @@ def test_row_range_fused_rejects_bad_ranges(begin, n):
                     ctypes.byref(cache), f0, 1, begin, n, FAKE, None, None)
     assert st == V.VMLA_ERR_INVALID_ARG and "token range" in d, d
 
+
+def test_ipc_calls_reject_bad_arguments():
+    """The CUDA IPC entry points validate their arguments before touching the driver: NULL handles or
+    pointers and releasing a pointer that vmla_ipc_import never returned are errors with a detail;
+    exporting an address that is not device memory fails cleanly (here: no GPU at all)."""
+    h = V.CIpcHandle()
+    st, d = _status(V.LIB.vmla_ipc_export, None, ctypes.byref(h))
+    assert st == V.VMLA_ERR_INVALID_ARG and "NULL" in d, d
+    st, d = _status(V.LIB.vmla_ipc_export, FAKE, None)
+    assert st == V.VMLA_ERR_INVALID_ARG, d
+    p = ctypes.c_void_p(0)
+    st, d = _status(V.LIB.vmla_ipc_import, None, ctypes.byref(p))
+    assert st == V.VMLA_ERR_INVALID_ARG, d
+    st, d = _status(V.LIB.vmla_ipc_release, FAKE)
+    assert st == V.VMLA_ERR_INVALID_ARG and "vmla_ipc_import" in d, d
+    st, d = _status(V.LIB.vmla_ipc_export, FAKE, ctypes.byref(h))
+    assert st != V.VMLA_OK, d
+
