@@ -485,3 +485,78 @@ def test_capacity_grows_as_the_latent_shrinks():
     caps = [O.batch_capacity(180 * 10**9, dense=False, **_wan_capacity_kwargs(d_c=d)) for d in (64, 128, 192)]
     dense = O.batch_capacity(180 * 10**9, dense=True, **_wan_capacity_kwargs())
     assert caps[0] > caps[1] > caps[2] > dense > 0
+
+
+def _weight_cases():
+    return [("wan", WAN), ("wan_dc64", WAN.replace(d_c=64)), ("tiny", TINY)]
+
+
+def _shape_kw(cfg):
+    return dict(dim=cfg.dim, n_heads=cfg.n_heads, d_nope=cfg.d_nope, d_rope=cfg.d_rope, d_c=cfg.d_c,
+                d_v=cfg.d_v)
+
+
+@pytest.mark.parametrize("name,cfg", _weight_cases())
+def test_layer_weights_are_the_drawn_weights(name, cfg):
+    """layer_weights lists exactly the tensors the seeded input recipe draws for one layer (shapes and
+    order: W^KV_down || W^KR, W^K_up, W^V_up; dense: the per-head K/V projection).  The recipe states
+    its shapes itself and holds none of the oracle's arithmetic, so a dropped weight, a missing head
+    axis or a d_nope / d_c swap in layer_weights fails here."""
+    drawn = synthetic.draw_weights(cfg, 7)
+    lw = O.layer_weights(dense=False, **_shape_kw(cfg))
+    assert [tuple(t.shape) for t in drawn] == list(lw.values())
+    dense = O.layer_weights(dense=True, **_shape_kw(cfg))
+    assert list(dense.values()) == [tuple(synthetic.draw_dense_weights(cfg, 7).shape)]
+
+
+@pytest.mark.parametrize("name,cfg", _weight_cases())
+def test_layer_weight_shapes_produce_the_printed_token_state(name, cfg):
+    """Weights of layer_weights' shapes, run through the oracle's own projections, give per token the
+    state the pages print: the stacked down-projection yields d_c + d_rope cached scalars (224 at the
+    defaults, Method item 4), the dense projection 2 n_h d_h scalars (3072), and the per-head keys and
+    values rebuilt from the latent have the dense head widths (d_nope + d_rope = d_h, and d_v)."""
+    rng = np.random.default_rng(3)
+    lw = O.layer_weights(dense=False, **_shape_kw(cfg))
+    w = {k: rng.standard_normal(v) for k, v in lw.items()}
+    T = 5
+    x = rng.standard_normal((T, cfg.dim))
+    pos = O.token_positions(0, T, cfg.grid_h, cfg.grid_w)
+    pairs = (cfg.rope_pairs_t, cfg.rope_pairs_h, cfg.rope_pairs_w)
+    c, k_r = O.compress(x, w["w_dkv_kr"], cfg.d_c, pos, pairs, cfg.rope_theta)
+    assert c.shape[-1] + k_r.shape[-1] == O.latent_scalars_per_token(cfg.d_c, cfg.d_rope)
+    k, v = O.reconstruct_kv(c, k_r, w["w_uk"], w["w_uv"])
+    assert k.shape == (T, cfg.n_heads, cfg.d_h) and v.shape == (T, cfg.n_heads, cfg.d_v)
+    q = O.absorbed_query(rng.standard_normal((T, cfg.n_heads, cfg.d_nope)),
+                         rng.standard_normal((T, cfg.n_heads, cfg.d_rope)), w["w_uk"])
+    assert q.shape == (T, cfg.n_heads, cfg.d_c + cfg.d_rope)
+    (rows, cols), = O.layer_weights(dense=True, **_shape_kw(cfg)).values()
+    assert cols == cfg.dim and rows == cfg.n_heads * (cfg.d_h + cfg.d_v)
+    if name == "wan":
+        g = json.load(open(GOLDEN))
+        assert c.shape[-1] + k_r.shape[-1] == 224
+        assert rows == 2 * g["n_heads"]["value"] * g["d_h"]["value"] == 3072
+
+
+@pytest.mark.parametrize("dense", [False, True])
+def test_memory_bytes_without_sequences_is_the_weights_and_fixed_bytes(dense):
+    """memory_bytes(0) holds no cache and no step tensor: it is n_layers times one layer's drawn
+    weights (counted from the seeded recipe's tensors) times the element size, plus the fixed bytes."""
+    for cfg, n_layers, fixed in ((WAN, 30, 0), (WAN.replace(d_c=64), 30, 12345), (TINY, 2, 1000)):
+        if dense:
+            numel = synthetic.draw_dense_weights(cfg, 1).numel()
+        else:
+            numel = sum(t.numel() for t in synthetic.draw_weights(cfg, 1))
+        kw = dict(n_layers=n_layers, window_tokens=cfg.window_tokens, elt_bytes=cfg.elt_bytes,
+                  fixed_bytes=fixed, extra_bytes_per_seq=777, tokens_per_chunk=cfg.chunk_tokens,
+                  **_shape_kw(cfg))
+        assert O.memory_bytes(0, dense=dense, **kw) == n_layers * numel * cfg.elt_bytes + fixed
+        # and one sequence adds its caches (every layer), its step tensors and its extra bytes
+        per_tok = cfg.dense_scalars_per_token() if dense else cfg.latent_scalars_per_token()
+        cache = n_layers * cfg.window_tokens * per_tok * cfg.elt_bytes
+        B, N, H = 1, cfg.chunk_tokens, cfg.n_heads
+        if dense:
+            step = N * cfg.dim + N * H * cfg.d_h + N * H * cfg.d_v
+        else:
+            step = N * cfg.dim + N * H * (cfg.d_nope + cfg.d_rope + cfg.d_v + cfg.d_c + cfg.d_rope + cfg.d_c)
+        assert O.memory_bytes(1, dense=dense, **kw) - O.memory_bytes(0, dense=dense, **kw) == \
+            cache + step * cfg.elt_bytes + 777
