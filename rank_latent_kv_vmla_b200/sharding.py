@@ -10,7 +10,16 @@ Per chunk, rank r
   2. waits, on the stream that carries the kernels, until every rank's rows are in place (a one-element
      all-reduce: it completes only after every rank's compress kernel has completed);
   3. advances frames_written of its replica records and attends with its own query rows
-     (vmla_latent_attention_fused_rows); attention itself needs no exchange.
+     (vmla_latent_attention_fused_rows); attention itself needs no exchange;
+  4. waits, again on the kernels' stream, until every rank's attention of this chunk has completed
+     (a second one-element all-reduce) before its next compress may start.
+
+Step 4 closes a write-after-read race between ranks: once the window is full, the next chunk's frames
+go to the ring slots of the oldest frames, and those frames are still inside this chunk's window.  A
+rank's compress writes into every replica, so without step 4 a rank that finished its attention early
+could overwrite rows that a slower rank's attention still reads.  With it, a replica is only ever
+written while no rank reads it: the compress of chunk k+1 on any rank is ordered after the attention of
+chunk k on every rank, and the attention of chunk k after the compress of chunk k on every rank.
 
 The communicator and the device operations are injectable (``comm``, ``ops``), so the protocol is
 exercised by multi-process CPU tests with stand-ins; on GPUs ``TorchComm`` (NCCL) and the library are
@@ -105,10 +114,13 @@ class ShardedLayer:
         for rep in self.replicas:
             rep.frames_written = f0 + cfg.chunk_frames
         self.cache.struct.frames_written = f0 + cfg.chunk_frames
-        if not self.count:
-            return None
-        return ops.latent_attention_fused_rows(cfg, q_nope_rows, q_rope_rows, w_uk, w_uv, self.cache, f0,
-                                               self.begin, out=out)
+        o = None
+        if self.count:
+            o = ops.latent_attention_fused_rows(cfg, q_nope_rows, q_rope_rows, w_uk, w_uv, self.cache, f0,
+                                                self.begin, out=out)
+        # no rank's next compress may overwrite ring rows before every rank has read this chunk's window
+        self.comm.device_barrier()
+        return o
 
     def close(self) -> None:
         """Unmap the peers' replicas once every rank is done with them."""

@@ -1,9 +1,13 @@
 """ShardedLayer end to end with two processes on one GPU (gloo process group): each rank exports its
 replica of the latent cache, imports the other's, compresses its token range of every chunk into both
 (through the CUDA IPC mapping), passes the device barrier (a gloo all-reduce of a device tensor, which
-completes only after both ranks' compress kernels) and attends with its own query rows on its own
-replica.  The ranks' output rows together must equal the unsharded fused call and the float64 oracle,
-and both replicas must equal the oracle's ring.  No kernel waits on the other process."""
+completes only after both ranks' compress kernels), attends with its own query rows on its own
+replica and passes the second device barrier (after both ranks' attention) before its next compress.
+Rank 0 sleeps on the host before every attention whose window the next chunk overwrites, so rank 1
+runs ahead as far as the protocol lets it: its next compress, which stores into rank 0's replica, must
+still wait for rank 0's attention.  The ranks' output rows together must equal the unsharded fused call
+and the float64 oracle, and both replicas must equal the oracle's ring.  No kernel waits on the other
+process."""
 import os
 import socket
 
@@ -33,6 +37,24 @@ def _unpack(a):
     return torch.from_numpy(a).view(torch.bfloat16)
 
 
+class _DelayedOps:
+    """The library calls as they are, except that rank 0 sleeps on the host before launching each
+    attention whose window the next chunk evicts frames of."""
+
+    def __init__(self, V, rank, delay_s=0.5):
+        self._V, self._rank, self._delay = V, rank, delay_s
+
+    def __getattr__(self, name):
+        return getattr(self._V, name)
+
+    def latent_attention_fused_rows(self, cfg, *args, **kw):
+        import time
+        f0 = args[5]
+        if self._rank == 0 and f0 + 2 * cfg.chunk_frames > cfg.window_frames:
+            time.sleep(self._delay)
+        return self._V.latent_attention_fused_rows(cfg, *args, **kw)
+
+
 def _rank(rank, world, port, q):
     import sys
     sys.path.insert(0, ROOT)
@@ -49,7 +71,7 @@ def _rank(rank, world, port, q):
         from parity import MID
         cfg, B = MID, 2
         torch.cuda.set_device(0)
-        layer = ShardedLayer(cfg, B, TorchComm(device="cuda"), device="cuda", align=8)
+        layer = ShardedLayer(cfg, B, TorchComm(device="cuda"), device="cuda", align=8, ops=_DelayedOps(V, rank))
         w, wuk, wuv = (t.cuda() for t in synthetic.draw_weights(cfg, 51))
         outs = []
         for k in range(N_CHUNKS):

@@ -1,13 +1,17 @@
 """Query-row sharding of one sequence (rank_latent_kv_vmla_b200.sharding) on the CPU.
 
 The host protocol runs in world-size-2 and world-size-3 gloo process groups with stand-ins for the
-device: a replica plane is a NumPy array; a store into another rank's replica is queued and delivered
-at the device barrier (which is where the real peer stores are known to have landed); compression and
-attention are the float64 oracle's.  After every streamed chunk each rank's replica must equal the
-oracle's ring, and the ranks' output rows together must equal the oracle's layer output."""
+device: a replica plane is a file-backed shared mapping (np.memmap), so a store into another rank's
+replica lands in that rank's memory at once, as a store through an NVLink peer mapping does;
+compression and attention are the float64 oracle's.  One rank is delayed on the host before every
+attention, so the other ranks run ahead as far as the protocol lets them.  Every rank's attention must
+see exactly the oracle's ring for its chunk, its output rows must equal the oracle's layer output, and
+after the last chunk every replica must equal the oracle's ring.  The same run with the release barrier
+after attention left out must see a peer overwrite rows that the delayed rank still reads."""
 import os
 import pickle
 import socket
+import time
 
 import numpy as np
 import pytest
@@ -41,9 +45,9 @@ def _free_port():
 
 
 class _Ptr:
-    """Stand-in device pointer: (owning rank, plane)."""
-    def __init__(self, owner, plane):
-        self.owner, self.plane = owner, plane
+    """Stand-in device pointer: (owning rank, plane) and the mapped array."""
+    def __init__(self, owner, plane, arr):
+        self.owner, self.plane, self.arr = owner, plane, arr
 
 
 class _Plane:
@@ -59,13 +63,25 @@ class _Struct:
         self.c, self.k_r, self.batch, self.frames_written = c, k_r, batch, frames_written
 
 
-class _Ops:
-    """CPU stand-in of the library calls ShardedLayer makes."""
+def _mapped(path, shape, create):
+    if create:
+        a = np.lib.format.open_memmap(path, mode="w+", dtype=np.float64, shape=shape)
+        a[...] = np.nan
+        a.flush()
+        return a
+    return np.lib.format.open_memmap(path, mode="r+")
 
-    def __init__(self, rank, O, pairs):
-        self.rank, self.O, self.pairs = rank, O, pairs
-        self.outbox = []
+
+class _Ops:
+    """CPU stand-in of the library calls ShardedLayer makes.  Replica planes live in shared file
+    mappings: a store into a peer's replica is visible to the peer immediately.  The rank
+    ``delay_rank`` sleeps ``delay_s`` before each attention whose window a later chunk overwrites."""
+
+    def __init__(self, rank, O, pairs, shm_dir, delay_rank=-1, delay_s=0.0):
+        self.rank, self.O, self.pairs, self.shm_dir = rank, O, pairs, shm_dir
+        self.delay_rank, self.delay_s = delay_rank, delay_s
         self.CCache = _Struct
+        self.seen = None
 
     def LatentCache(self, cfg, batch, device=None):
         rank = self.rank
@@ -73,8 +89,9 @@ class _Ops:
         class _Cache:
             pass
         cache = _Cache()
-        cache.c = _Plane(np.full((batch, cfg.window_tokens, cfg.d_c), np.nan), _Ptr(rank, "c"))
-        cache.k_r = _Plane(np.full((batch, cfg.window_tokens, cfg.d_rope), np.nan), _Ptr(rank, "k_r"))
+        for plane, d in (("c", cfg.d_c), ("k_r", cfg.d_rope)):
+            arr = _mapped(os.path.join(self.shm_dir, f"r{rank}_{plane}.npy"), (batch, cfg.window_tokens, d), True)
+            setattr(cache, plane, _Plane(arr, _Ptr(rank, plane, arr)))
         cache.struct = _Struct(cache.c.data_ptr(), cache.k_r.data_ptr(), batch, 0, 0)
         cache.batch = batch
         type(cache).frames_written = property(lambda s: s.struct.frames_written)
@@ -88,16 +105,11 @@ class _Ops:
     def ipc_import(self, handle):
         owner, plane = pickle.loads(handle)
         assert owner != self.rank
-        return _Ptr(owner, plane)
+        return _Ptr(owner, plane, _mapped(os.path.join(self.shm_dir, f"r{owner}_{plane}.npy"), None, False))
 
     def ipc_release(self, ptr):
         assert ptr.owner != self.rank
-
-    def _store(self, ptr, b, rows, vals):
-        if ptr.owner == self.rank:
-            getattr(self.local, ptr.plane).arr[b, rows] = vals
-        else:
-            self.outbox.append((ptr.owner, ptr.plane, b, rows, vals))
+        ptr.arr.flush()
 
     def compress_append_rows(self, cfg, x_rows, w, f0, begin, replicas, batch):
         O = self.O
@@ -110,17 +122,14 @@ class _Ops:
             assert r.frames_written == f0
         for b in range(batch):
             c, k_r = O.compress(x_rows[b], w, cfg.d_c, pos, self.pairs, cfg.rope_theta)
-            for r in replicas:
-                self._store(r.c, b, rows, c)
-                self._store(r.k_r, b, rows, k_r)
-
-    def deliver(self, incoming):
-        for owner, plane, b, rows, vals in incoming:
-            assert owner == self.rank
-            getattr(self.local, plane).arr[b, rows] = vals
+            for r in replicas:                      # stores land in the target replica at once
+                r.c.arr[b, rows] = c
+                r.k_r.arr[b, rows] = k_r
 
     def latent_attention_fused_rows(self, cfg, qn, qr, w_uk, w_uv, cache, f0, begin, out=None):
         O = self.O
+        if self.rank == self.delay_rank and f0 + 2 * cfg.chunk_frames > cfg.window_frames:
+            time.sleep(self.delay_s)                # the next chunk evicts frames of this window
         n = qn.shape[1]
         fw = cache.frames_written
         key_frames = np.repeat([O.frame_of_slot(s, fw, cfg.window_frames) for s in range(cfg.window_frames)],
@@ -128,23 +137,29 @@ class _Ops:
         pos = O.token_positions(f0, cfg.chunk_tokens, cfg.grid_h, cfg.grid_w)[begin:begin + n]
         hi = O.query_chunk_end(f0, cfg.chunk_tokens, cfg.chunk_frames, cfg.tokens_per_frame)[begin:begin + n]
         mask = O.visible(hi, key_frames, cfg.window_frames) & (key_frames >= 0)[None, :]
+        self.seen = (np.array(cache.c.arr), np.array(cache.k_r.arr))     # what this attention reads
         outs = []
         for b in range(qn.shape[0]):
             q_abs = O.absorbed_query(qn[b], O.rotate_query(qr[b], pos, self.pairs, cfg.rope_theta), w_uk)
-            c = np.nan_to_num(cache.c.arr[b])
-            k_r = np.nan_to_num(cache.k_r.arr[b])
+            c = np.nan_to_num(self.seen[0][b])
+            k_r = np.nan_to_num(self.seen[1][b])
             o_lat, _ = O.latent_attention(q_abs, c, k_r, mask, cfg.scale)
             outs.append(O.value_up(o_lat, w_uv))
         return np.stack(outs)
 
 
 class _Comm:
-    """gloo collectives; queued peer stores are delivered at the device barrier."""
+    """gloo collectives.  The device barrier is a host all-reduce: the stand-in's stores are made
+    synchronously, so every store issued before it has landed when it returns.  ``release_barrier``
+    False turns every second device barrier (the one after attention) into a no-op on every rank."""
 
-    def __init__(self, dist, ops):
-        self.dist, self.ops = dist, ops
+    def __init__(self, dist, release_barrier=True):
+        import torch
+        self.dist, self.torch = dist, torch
         self.world, self.rank = dist.get_world_size(), dist.get_rank()
+        self.release_barrier = release_barrier
         self.n_barriers = 0
+        self._calls = 0
 
     def all_gather_object(self, obj):
         out = [None] * self.world
@@ -152,21 +167,23 @@ class _Comm:
         return out
 
     def device_barrier(self):
-        boxes = self.all_gather_object(self.ops.outbox)
-        self.ops.outbox = []
-        self.ops.deliver([m for box in boxes for m in box if m[0] == self.rank])
+        self._calls += 1
+        if not self.release_barrier and self._calls % 2 == 0:
+            return
+        self.dist.all_reduce(self.torch.zeros(1))
         self.n_barriers += 1
 
     def barrier(self):
         self.dist.barrier()
 
 
-def _worker(rank, world, port, root, q):
+def _worker(rank, world, port, root, shm_dir, release_barrier, q):
     import sys
     sys.path.insert(0, root)
     os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    import datetime
     import torch.distributed as dist
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
     try:
         from oracle import vmla_oracle as O
         from rank_latent_kv_vmla_b200.config import TINY
@@ -174,14 +191,14 @@ def _worker(rank, world, port, root, q):
         import synthetic
         cfg = TINY.replace(grid_h=4, grid_w=6, chunk_frames=1, window_frames=3)     # 24 tokens per chunk
         pairs = (cfg.rope_pairs_t, cfg.rope_pairs_h, cfg.rope_pairs_w)
-        ops = _Ops(rank, O, pairs)
-        comm = _Comm(dist, ops)
+        ops = _Ops(rank, O, pairs, shm_dir, delay_rank=0, delay_s=0.4)
+        comm = _Comm(dist, release_barrier)
         B, n_chunks = 2, 5
         layer = ShardedLayer(cfg, B, comm, ops=ops, align=8)
         w = synthetic.draw_weights(cfg, 5)
         w, w_uk, w_uv = (t.double().numpy() for t in w)
         hists = [O.History(cfg.d_c, cfg.d_rope) for _ in range(B)]
-        report = []
+        report, seen_err, out_err = [], 0.0, 0.0
         for k in range(n_chunks):
             x, qn, qr = (t.double().numpy() for t in synthetic.draw_chunk(cfg, B, 50 + k))
             f0 = layer.frames_written
@@ -191,44 +208,73 @@ def _worker(rank, world, port, root, q):
             for b in range(B):
                 c, k_r = O.compress(x[b], w, cfg.d_c, pos, pairs, cfg.rope_theta)
                 hists[b].append(c, k_r, pos[:, 0])
-            for b in range(B):
-                c_ref, written = O.ring_from_history(hists[b].c, layer.frames_written, cfg.window_frames,
-                                                     cfg.tokens_per_frame)
-                kr_ref, _ = O.ring_from_history(hists[b].k_r, layer.frames_written, cfg.window_frames,
-                                                cfg.tokens_per_frame)
-                np.testing.assert_allclose(ops.local.c.arr[b][written], c_ref[written], rtol=0, atol=1e-12)
-                np.testing.assert_allclose(ops.local.k_r.arr[b][written], kr_ref[written], rtol=0, atol=1e-12)
-                assert np.isnan(ops.local.c.arr[b][~written]).all()
-            # this rank's output rows against the oracle's whole-layer reference
             if cnt:
+                # the replica this rank's attention read, and its output rows, against the oracle
                 for b in range(B):
+                    for plane, hist in ((0, hists[b].c), (1, hists[b].k_r)):
+                        ref, written = O.ring_from_history(hist, layer.frames_written, cfg.window_frames,
+                                                           cfg.tokens_per_frame)
+                        got = ops.seen[plane][b]
+                        seen_err = max(seen_err, float(np.nan_to_num(np.abs(got[written] - ref[written]),
+                                                                     nan=np.inf).max()))
+                        assert np.isnan(got[~written]).all()
                     ref = O.layer_reference(hists[b], qn[b], qr[b], w_uk, w_uv, first_frame=f0,
                                             query_rows=np.arange(b0, b0 + cnt), chunk_frames=cfg.chunk_frames,
                                             window_frames=cfg.window_frames, grid_h=cfg.grid_h,
                                             grid_w=cfg.grid_w, pairs=pairs, theta=cfg.rope_theta, scale=cfg.scale)
-                    np.testing.assert_allclose(o[b], ref["o"], rtol=1e-10, atol=1e-12)
+                    out_err = max(out_err, float(np.abs(o[b] - ref["o"]).max()))
             report.append((k, b0, cnt, layer.frames_written))
         layer.close()
-        q.put((rank, report, comm.n_barriers, [r.frames_written for r in layer.replicas]))
+        # after the last chunk (close() holds two barriers) every replica equals the oracle's ring
+        final_err = 0.0
+        for b in range(B):
+            for arr, hist in ((ops.local.c.arr, hists[b].c), (ops.local.k_r.arr, hists[b].k_r)):
+                ref, written = O.ring_from_history(hist, layer.frames_written, cfg.window_frames,
+                                                   cfg.tokens_per_frame)
+                final_err = max(final_err, float(np.abs(arr[b][written] - ref[written]).max()))
+        q.put((rank, report, comm.n_barriers, [r.frames_written for r in layer.replicas],
+               seen_err, out_err, final_err))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_sharded_layer_protocol_gloo(repo_root, world):
+def _run(world, tmp_path, release_barrier):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, repo_root, q)) for r in range(world)]
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    procs = [ctx.Process(target=_worker, args=(r, world, port, root, str(tmp_path), release_barrier, q))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
         p.join(timeout=300)
         assert p.exitcode == 0
-    got = sorted(q.get(timeout=5) for _ in range(world))
+    return sorted(q.get(timeout=5) for _ in range(world))
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_layer_protocol_gloo(world, tmp_path):
+    """Rank 0 is delayed before every attention; the other ranks' next compress must still wait."""
+    got = _run(world, tmp_path, release_barrier=True)
     shards = token_shards(24, world, 8)
-    for rank, report, n_barriers, replica_frames in got:
-        assert n_barriers == 5                          # one device barrier per chunk on every rank
+    for rank, report, n_barriers, replica_frames, seen_err, out_err, final_err in got:
+        assert n_barriers == 2 * 5                      # two device barriers per chunk on every rank
         assert replica_frames == [5] * world
         assert [(b, c) for _, b, c, _ in report] == [shards[rank]] * 5
-        assert [f for *_, f in report] == [1, 2, 3, 4, 5]
+        assert [f for *_, f in report][:5] == [1, 2, 3, 4, 5]
+        assert seen_err <= 1e-12, (rank, seen_err)      # the attention read exactly the oracle's ring
+        assert out_err <= 1e-10, (rank, out_err)
+        assert final_err <= 1e-12, (rank, final_err)
+
+
+def test_without_the_release_barrier_a_peer_overwrites_a_window_in_use(tmp_path):
+    """The protocol with only the barrier after the compress: while rank 0 sleeps before its attention,
+    rank 1 compresses the next chunk into rank 0's replica, evicting frames of the window rank 0 is
+    about to read.  The stand-ins detect it (this is the race the release barrier closes)."""
+    got = _run(2, tmp_path, release_barrier=False)
+    seen_err = {rank: e for rank, _, _, _, e, _, _ in got}
+    out_err = {rank: e for rank, _, _, _, _, e, _ in got}
+    assert seen_err[0] > 1e-3 and out_err[0] > 1e-6
+    # the rank that is never delayed reads correct windows (nobody writes into its window early)
+    assert seen_err[1] <= 1e-12
