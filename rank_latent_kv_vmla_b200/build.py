@@ -3,6 +3,11 @@
     python -m rank_latent_kv_vmla_b200.build [--force] [--jobs N] [--checked]
 
 Objects go to ``_build/`` at the repository root; the shared library is written next to this file.
+Whether an object or the library is current is decided by content, not by modification times: each
+object records a SHA-256 of its source, every header, this script and the compiler flags, and the
+library records the hashes of the objects it was linked from (``<lib>.sha256``).  A build whose
+recorded hash differs, or is missing, is redone, so objects or libraries carried over from another
+checkout are never used as they are.
 ``--checked`` builds ``libvmla_checked.so`` (objects in ``_build_checked/``) with VMLA_CHECKED=1: every
 computed global store of the tensor-core kernels is tested against its buffer's extent (a store outside
 is skipped and reported in the device status word).  Select it with VMLA_LIBRARY=<path> at import.
@@ -12,6 +17,7 @@ from __future__ import annotations
 import argparse
 import concurrent.futures as cf
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -42,11 +48,44 @@ def _headers():
     return glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def _stale(target: str, deps) -> bool:
-    if not os.path.exists(target):
-        return True
-    t = os.path.getmtime(target)
-    return any(os.path.getmtime(d) > t for d in deps)
+def _flags_key(flags) -> list:
+    """The compiler flags without this checkout's paths (a checkout elsewhere hashes the same), plus the
+    compiler's version."""
+    rel = [os.path.relpath(f, ROOT) if os.path.isabs(f) else f for f in flags]
+    return rel + [_nvcc_version()]
+
+
+_NVCC_VERSION = []
+
+
+def _nvcc_version() -> str:
+    if not _NVCC_VERSION:
+        r = subprocess.run([nvcc(), "--version"], capture_output=True, text=True)
+        _NVCC_VERSION.append(r.stdout.strip().splitlines()[-1] if r.returncode == 0 and r.stdout.strip() else "")
+    return _NVCC_VERSION[0]
+
+
+def _digest(paths, extra) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(os.path.basename(p).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    h.update(repr(list(extra)).encode())
+    return h.hexdigest()
+
+
+def _recorded(target: str) -> str:
+    try:
+        with open(target + ".sha256") as f:
+            return f.read().strip()
+    except OSError:
+        return ""
+
+
+def _record(target: str, digest: str) -> None:
+    with open(target + ".sha256", "w") as f:
+        f.write(digest + "\n")
 
 
 def _compile(src: str, obj: str, extra):
@@ -63,25 +102,31 @@ def build(force: bool = False, jobs: int = 0, extra=(), verbose: bool = False, c
     os.makedirs(build_dir, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = _headers()
-    objs, todo = [], []
+    objs, todo, digests = [], [], []
+    common = sorted(headers) + [os.path.abspath(__file__)]
     for src in sources:
         obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
+        digest = _digest([src] + common, _flags_key(NVCC_FLAGS + list(extra)))
         objs.append(obj)
-        if force or _stale(obj, [src] + headers + [__file__]):
-            todo.append((src, obj))
+        digests.append(digest)
+        if force or not os.path.exists(obj) or _recorded(obj) != digest:
+            todo.append((src, obj, digest))
     if todo:
         n = jobs or min(len(todo), os.cpu_count() or 1)
         with cf.ThreadPoolExecutor(max_workers=n) as ex:
-            for (src, _), log in zip(todo, ex.map(lambda so: _compile(so[0], so[1], extra), todo)):
+            for (src, obj, digest), log in zip(todo, ex.map(lambda t: _compile(t[0], t[1], extra), todo)):
+                _record(obj, digest)
                 if verbose and log:
                     print(f"--- {os.path.basename(src)}\n{log}", file=sys.stderr)
-    if force or todo or _stale(lib, objs):
+    lib_digest = hashlib.sha256("".join(digests).encode()).hexdigest()
+    if force or todo or not os.path.exists(lib) or _recorded(lib) != lib_digest:
         tmp = lib + ".tmp"
         cmd = [nvcc(), "-shared", "-o", tmp] + objs + ARCH
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
         os.replace(tmp, lib)
+        _record(lib, lib_digest)
     return lib
 
 
