@@ -240,7 +240,9 @@ VMLA_API vmla_status vmla_check_fused(const vmla_config* cfg);
 
 /* Synchronise `stream`, then read and clear the device status word of the current device:
  * *code = 0 if no device-side wait ran out since the last call, else a nonzero code naming the wait.
- * Returns VMLA_ERR_TIMEOUT when *code != 0. */
+ * The read and the clear are one atomic exchange made by a one-thread kernel on `stream`, so a code
+ * that a kernel on another stream raises meanwhile is either returned by this call or kept for the
+ * next one, never lost.  Returns VMLA_ERR_TIMEOUT when *code != 0. */
 VMLA_API vmla_status vmla_device_status(void* stream, int32_t* code);
 
 /* Bytes of one layer's cache for `batch` sequences at a full window: latent (d_c + d_rope per token)
@@ -288,7 +290,10 @@ VMLA_API vmla_status vmla_plan_capacity(const vmla_config* cfg, int32_t n_layers
  * stay the caller's; the executor owns only its two streams and six events.  Host buffers should be
  * page-locked (pageable memory makes the copies synchronous); an input buffer may be reused, and
  * out_host read, only after vmla_executor_wait().  cache->frames_written advances at submit.
- * bf16 only (VMLA_ERR_UNSUPPORTED otherwise); errors of the inner calls are returned as they are. */
+ * bf16 only (VMLA_ERR_UNSUPPORTED otherwise); errors of the inner calls are returned as they are.
+ * A submit refused on the host (null or misaligned pointers, an unsupported shape) enqueues nothing and
+ * leaves the cache and the executor as they were; only a CUDA error after the step's compress was
+ * enqueued leaves frames_written advanced (the chunk's rows are then in the ring). */
 typedef struct vmla_executor vmla_executor;
 VMLA_API int64_t vmla_executor_workspace_bytes(const vmla_config* cfg, int32_t batch);   /* -1 on bad args */
 VMLA_API vmla_status vmla_executor_create(const vmla_config* cfg, int32_t batch, void* workspace,

@@ -17,6 +17,12 @@ thread_local std::string g_detail;
 std::atomic<int64_t> g_launches{0};
 
 __device__ int g_device_status;
+__device__ int g_status_taken;   // the value vmla_device_status last swapped out of g_device_status
+
+// Read and clear the status word in one atomic step, so that a code a kernel on another stream raises
+// at any moment is either returned now or kept for the next read.
+__global__ void take_status_kernel() { g_status_taken = atomicExch(&g_device_status, 0); }
+std::mutex g_take_mu;
 
 constexpr int kMaxDevices = 64;
 int* g_status_addr[kMaxDevices];
@@ -615,16 +621,20 @@ vmla_status vmla_check_fused(const vmla_config* cfg) {
 
 vmla_status vmla_device_status(void* stream, int32_t* code) {
   if (!code) return fail(VMLA_ERR_INVALID_ARG, "code is NULL");
-  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  cudaStream_t st = as_stream(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
-  int* p = device_status_ptr();
-  if (!p) return fail(VMLA_ERR_CUDA, "cannot resolve the device status word");
+  if (!device_status_ptr()) return fail(VMLA_ERR_CUDA, "cannot resolve the device status word");
   int v = 0;
-  e = cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost);
+  {
+    std::lock_guard<std::mutex> lk(g_take_mu);      // one swap-and-read at a time per process
+    take_status_kernel<<<1, 1, 0, st>>>();
+    count_launches(1);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbolAsync(&v, g_status_taken, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "read device status");
-  const int zero = 0;
-  e = cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
-  if (e != cudaSuccess) return cuda_fail(e, "clear device status");
   *code = v;
   if (v != 0) return fail(VMLA_ERR_TIMEOUT, "device wait %d ran out", v);
   return VMLA_OK;

@@ -93,6 +93,18 @@ vmla_status vmla_executor_submit(vmla_executor* ex, vmla_cache* cache, const voi
   if (!ex || !cache || !x_host || !q_nope_host || !q_rope_host || !out_host)
     return vmla::report(VMLA_ERR_INVALID_ARG, "executor, cache and host buffers must not be NULL");
   if (cache->batch != ex->batch) return vmla::report(VMLA_ERR_INVALID_ARG, "cache batch differs from the executor's");
+  // everything the two calls below check on the host is checked here first, so that a refused step
+  // enqueues nothing: no copy, no compress (which would advance frames_written and evict a frame)
+  for (const void* p : {(const void*)cache->c, (const void*)cache->k_r, w_dkv_kr, w_uk, w_uv}) {
+    if (!p) return vmla::report(VMLA_ERR_INVALID_ARG, "cache planes and weights must not be NULL");
+    if (reinterpret_cast<uintptr_t>(p) & 15u)
+      return vmla::report(VMLA_ERR_MISALIGNED, "cache planes and weights must be 16-byte aligned");
+  }
+  vmla_status chk = vmla_check_fused(&ex->cfg);
+  if (chk != VMLA_OK) return chk;
+  chk = vmla_check_attention_window(&ex->cfg, cache->frames_written + ex->cfg.chunk_frames,
+                                    cache->frames_written, 1);
+  if (chk != VMLA_OK) return chk;
   const int s = (int)(ex->submitted % kSlots);
   uint8_t* x = ex->slot[s];
   uint8_t* qn = x + round_up(ex->sz.x);

@@ -66,7 +66,20 @@ def test_executor_rejects_bad_submissions(V):
         with pytest.raises(ValueError):
             ex.submit(V.LatentCache(cfg, 2, device=DEV), w, wuk, wuv, x.cuda(), qn, qr, ho)   # device input
         cache = V.LatentCache(cfg, 2, device=DEV)
+        # refused on the host by a check of the inner fused call (a misaligned W^V_up): nothing is
+        # enqueued, the cache is not advanced and no ring row is written
+        import ctypes
+        st = V.LIB.vmla_executor_submit(ex._h, ctypes.byref(cache.struct), w.data_ptr(), wuk.data_ptr(),
+                                        wuv.data_ptr() + 2, x.data_ptr(), qn.data_ptr(), qr.data_ptr(),
+                                        ho.data_ptr())
+        assert st == V.VMLA_ERR_MISALIGNED
+        assert cache.frames_written == 0
         ex.submit(cache, w, wuk, wuv, x, qn, qr, ho)          # the executor still works afterwards
         ex.wait()
         assert cache.frames_written == cfg.chunk_frames
+        ref = V.LatentCache(cfg, 2, device=DEV)
+        o_ref = V.layer_step(cfg, x.to(DEV), qn.to(DEV), qr.to(DEV), w, wuk, wuv, ref, fused=True).cpu()
+        assert torch.equal(ho, o_ref)
+        n = cfg.chunk_tokens                                  # the rows of frames 0 .. F-1
+        assert torch.equal(ref.c[:, :n], cache.c[:, :n]) and torch.equal(ref.k_r[:, :n], cache.k_r[:, :n])
     assert V.device_status() == 0
