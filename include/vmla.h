@@ -324,6 +324,15 @@ VMLA_API void vmla_debug_drop_kv_tile(int32_t tile);
  * 0 clears it.  Returns 1 in a checked build, 0 otherwise (where the hook has no effect). */
 VMLA_API int32_t vmla_debug_shrink_extents(int64_t bytes);
 
+/* Test hook of the exponential that the bf16 attention kernels compute on the FMA pipe for part of
+ * their softmax terms (the rest use the MUFU ex2 unit).  Its method: x = n + f with n the nearest
+ * integer, 2^f from a cubic fitted for least maximum relative error on [-1/2, 1/2] (Lawson's
+ * iteration), n added to the exponent field; arguments below -125 are clamped to -125.  Claimed
+ * accuracy: relative error <= 7.5e-5 for -125 <= x <= 120, and 2^-125 within that error for x < -125,
+ * -inf and NaN.  y[i] = that 2^x of x[i], i < n: x and y are device buffers of n floats; the kernel
+ * runs on `stream`.  VMLA_ERR_INVALID_ARG on NULL pointers or n < 0. */
+VMLA_API vmla_status vmla_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream);
+
 /* Number of kernels the library has launched in this process (all entry points, all devices). */
 VMLA_API int64_t vmla_launch_count(void);
 

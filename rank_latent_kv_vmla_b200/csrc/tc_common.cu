@@ -4,8 +4,9 @@
 #include <atomic>
 #include <mutex>
 
+#include "ptx_sm100.cuh"
 #include "tc_common.cuh"
-#include "vmla.h"
+#include "vmla_internal.cuh"
 
 namespace vmla {
 namespace {
@@ -91,4 +92,33 @@ extern "C" VMLA_API void vmla_debug_drop_kv_tile(int32_t tile) { vmla::g_drop_kv
 extern "C" VMLA_API int32_t vmla_debug_shrink_extents(int64_t bytes) {
   vmla::g_shrink_extents.store(bytes > 0 ? bytes : 0);
   return VMLA_CHECKED;
+}
+
+namespace vmla {
+namespace {
+// One pair of arguments per thread through exactly the device function the softmax warps call.
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  const int64_t stride = 2 * (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < n; i += stride) {
+    const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : 0.f;
+    float y0, y1;
+    sm100::exp2_poly2(y0, y1, x0, x1);
+    y[i] = y0;
+    if (i + 1 < n) y[i + 1] = y1;
+  }
+}
+}  // namespace
+}  // namespace vmla
+
+extern "C" VMLA_API vmla_status vmla_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+  if (!x || !y || n < 0) return vmla::report(VMLA_ERR_INVALID_ARG, "x and y must not be NULL and n >= 0");
+  if (n == 0) return VMLA_OK;
+  const int64_t pairs = (n + 1) / 2;
+  const int threads = 256;
+  const int64_t want = (pairs + threads - 1) / threads;
+  const int blocks = (int)(want < 148 * 8 ? want : 148 * 8);
+  vmla::exp2_poly_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  vmla::count_launches(1);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? VMLA_OK : vmla::report(VMLA_ERR_CUDA, cudaGetErrorString(e));
 }

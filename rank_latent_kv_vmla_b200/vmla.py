@@ -35,7 +35,7 @@ EXPORTED = ("vmla_compress_append", "vmla_absorb_q", "vmla_latent_attention", "v
             "vmla_latent_attention_fused", "vmla_executor_workspace_bytes", "vmla_executor_create",
             "vmla_executor_submit", "vmla_executor_wait", "vmla_executor_destroy",
             "vmla_compress_append_rows", "vmla_latent_attention_fused_rows", "vmla_ipc_export",
-            "vmla_ipc_import", "vmla_ipc_release", "vmla_debug_shrink_extents")
+            "vmla_ipc_import", "vmla_ipc_release", "vmla_debug_shrink_extents", "vmla_debug_exp2_poly")
 
 
 class VmlaError(RuntimeError):
@@ -103,6 +103,7 @@ def _load():
         "vmla_executor_submit": [VP, P(CCache), VP, VP, VP, VP, VP, VP, VP],
         "vmla_executor_wait": [VP],
         "vmla_executor_destroy": [VP],
+        "vmla_debug_exp2_poly": [VP, VP, I64, VP],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -441,6 +442,15 @@ def debug_drop_kv_tile(tile: int) -> None:
     """Test hook: the next bf16 latent attention launch skips loading KV tile ``tile`` (its wait runs
     out and vmla_device_status reports it); tile < 0 clears the request."""
     LIB.vmla_debug_drop_kv_tile(int(tile))
+
+
+def debug_exp2_poly(x: torch.Tensor) -> torch.Tensor:
+    """Test hook: the FMA-pipe 2^x of the attention kernels' softmax, applied to a float32 CUDA tensor."""
+    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    check(LIB.vmla_debug_exp2_poly(x.data_ptr(), y.data_ptr(), x.numel(), _stream(x)))
+    return y
 
 
 def launch_count() -> int:

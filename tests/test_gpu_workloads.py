@@ -1,6 +1,7 @@
 """GPU parity at the full sizes of the larger workloads: the Wan-1.3B layer at batch 8 with the dense
 per-head layer on identical inputs, the lower-rank latents at batch 16, and a long streaming rollout
-whose ring wraps many times (frame indices up to 240).  The oracle checks sampled query rows of batch
+whose ring wraps many times (frame indices up to 240).  At batch 8 and 16 both the three-call path and
+the fused call (the one the bench times there) are checked.  The oracle checks sampled query rows of batch
 elements {0, B-1} and whole cache planes; the dense and latent paths are also compared in full."""
 import numpy as np
 import pytest
@@ -9,7 +10,7 @@ import torch
 from oracle import vmla_oracle as O
 from rank_latent_kv_vmla_b200.config import WAN
 import synthetic
-from parity import OracleLayer, assert_close, dense_weights_from_latent, f64, round_to, pairs
+from parity import OracleLayer, assert_close, dense_weights_from_latent, errors, f64, round_to, pairs
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -50,11 +51,15 @@ def test_wan_batch8_latent_and_dense_agree_with_oracle(V):
     o_lat = V.latent_attention(cfg, V.absorb_q(cfg, qn, qr, _to(inp.w_uk), f0), lc, f0)
     o_l = V.value_up(cfg, o_lat, _to(inp.w_uv))
     o_d = V.dense_mha(cfg, V.rope_q(cfg, qn, qr, f0), dc, f0)
+    # the fused call (absorb + attention + value-up in one launch), as the batch-8 bench times it
+    o_f, lse_f = V.latent_attention_fused(cfg, qn, qr, _to(inp.w_uk), _to(inp.w_uv), lc, f0, want_lse=True)
     torch.cuda.synchronize()
     assert V.device_status() == 0
-    # both paths, all rows, against each other
+    # the paths, all rows, against each other
     for b in range(B):
         assert_close(f64(o_d[b]), f64(o_l[b]), cfg, f"dense vs latent b{b}")
+        rel_l2, max_ratio = errors(f64(o_f[b]), f64(o_l[b]))
+        assert rel_l2 <= 2e-3 and max_ratio <= 1e-2, (b, rel_l2, max_ratio)
     # and sampled rows of the first and last sequence against the oracle
     orc = OracleLayer(cfg, inp, B)
     rows = _rows(cfg)
@@ -63,6 +68,8 @@ def test_wan_batch8_latent_and_dense_agree_with_oracle(V):
     for b in (0, B - 1):
         ref = orc.reference(b, inp.q_nope, inp.q_rope, f0, rows=rows)
         assert_close(f64(o_l[b][rows]), ref["o"], cfg, f"latent o b{b}")
+        assert_close(f64(o_f[b][rows]), ref["o"], cfg, f"fused o b{b}")
+        assert_close(f64(lse_f[b][rows]), ref["lse"], cfg, f"fused lse b{b}")
         assert_close(f64(o_d[b][rows]), ref["o"], cfg, f"dense o b{b}")
         c_ref, kr_ref, written = orc.ring(b)
         assert written.all()
@@ -81,9 +88,18 @@ def test_wan_lower_rank_batch16(V, d_c):
     q_abs = V.absorb_q(cfg, _to(inp.q_nope), _to(inp.q_rope), _to(inp.w_uk), f0)
     o_lat, lse = V.latent_attention(cfg, q_abs, cache, f0, want_lse=True)
     o = V.value_up(cfg, o_lat, _to(inp.w_uv))
+    # the fused call, as the d_c sweep of the bench times it at this batch
+    fused = V.fused_supported(cfg)
+    assert fused or d_c == 64
+    if fused:
+        o_f, lse_f = V.latent_attention_fused(cfg, _to(inp.q_nope), _to(inp.q_rope), _to(inp.w_uk),
+                                              _to(inp.w_uv), cache, f0, want_lse=True)
     torch.cuda.synchronize()
     assert V.device_status() == 0
     assert cache.nbytes() == V.latent_cache_bytes(cfg, B)
+    for b in range(B if fused else 0):
+        rel_l2, max_ratio = errors(f64(o_f[b]), f64(o[b]))
+        assert rel_l2 <= 2e-3 and max_ratio <= 1e-2, (b, rel_l2, max_ratio)
     orc = OracleLayer(cfg, inp, B)
     for x in inp.x_chunks:
         orc.append(x)
@@ -93,6 +109,9 @@ def test_wan_lower_rank_batch16(V, d_c):
         assert_close(f64(o_lat[b][rows]), ref["o_latent"], cfg, f"o_latent b{b}")
         assert_close(f64(lse[b][rows]), ref["lse"], cfg, f"lse b{b}")
         assert_close(f64(o[b][rows]), ref["o"], cfg, f"o b{b}")
+        if fused:
+            assert_close(f64(o_f[b][rows]), ref["o"], cfg, f"fused o b{b}")
+            assert_close(f64(lse_f[b][rows]), ref["lse"], cfg, f"fused lse b{b}")
 
 
 def test_streaming_rollout_80_chunks(V):
