@@ -141,13 +141,28 @@ def source_hash(names):
 # ------------------------------------------------------------------------------------------------
 # Clock sampling during the timed region
 # ------------------------------------------------------------------------------------------------
+_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+def gpu_bus_id(cuda_index: int):
+    """PCI bus id of a CUDA device, as NVML and nvidia-smi name it (CUDA and NVML may order devices
+    differently); None if torch does not report it."""
+    try:
+        pr = torch.cuda.get_device_properties(cuda_index)
+        return "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+    except Exception:
+        return None
+
+
 class ClockSampler:
+    """nvidia-smi every 100 ms in a child process: the clocks line of the whole measured run (timed
+    region, interleaved path comparison, end-to-end leg, sustained leg)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+        self.gpu = gpu_bus_id(gpu_index) or str(gpu_index)
         self.proc = None
         self.path = None
 
@@ -156,11 +171,38 @@ class ClockSampler:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.out = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.out, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+
+    @staticmethod
+    def _parse(lines):
+        sm, smax, reasons = [], None, set()
+        for line in lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(_REASONS, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return sm, smax, reasons
+
+    def snapshot(self):
+        """One blocking nvidia-smi sample (parsed), or None."""
+        try:
+            r = subprocess.run(["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                                "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=20)
+            sm, smax, reasons = self._parse(r.stdout.splitlines())
+            return {"sm_mhz": sm[0], "sm_max_mhz": smax, "reasons": sorted(reasons)} if sm else None
+        except Exception:
+            return None
 
     def stop(self):
         if self.proc is None:
@@ -171,25 +213,76 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.out.close()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
+        sm, smax, reasons = self._parse(open(self.path))
         os.unlink(self.path)
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi every 100 ms"}
+
+
+class NvmlSampler:
+    """SM clock and clock-event reasons read through NVML every ``period_s`` by a host thread, so that
+    even a timed region of a few tens of milliseconds holds samples.  mark() opens a named window;
+    window(name) summarises the samples taken in it."""
+    _BITS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+             "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, cuda_index: int, period_s: float = 0.002):
+        import threading
+        self.period = period_s
+        self.samples = []             # (t, sm_mhz, reasons bitmask)
+        self.marks = {}
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            bus = gpu_bus_id(cuda_index)
+            self.h = (pynvml.nvmlDeviceGetHandleByPciBusId(bus) if bus
+                      else pynvml.nvmlDeviceGetHandleByIndex(cuda_index))
+            self.nv = pynvml
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.nv = None
+
+    def start(self):
+        if self.nv is None:
+            return
+        import threading
+
+        def loop():
+            nv, h = self.nv, self.h
+            while not self._stop.is_set():
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((time.perf_counter(), float(mhz), int(rs)))
+                except Exception:
+                    pass
+                time.sleep(self.period)
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+
+    def mark(self, name: str, end: bool = False):
+        self.marks.setdefault(name, [None, None])[1 if end else 0] = time.perf_counter()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+
+    def window(self, name: str):
+        t0, t1 = self.marks.get(name, (None, None))
+        if t0 is None or t1 is None:
+            return None
+        got = [(mhz, rs) for t, mhz, rs in self.samples if t0 <= t <= t1]
+        if not got:
+            return None
+        reasons = sorted(n for n, bit in self._BITS.items() if any(rs & bit for _, rs in got))
+        return {"sm_mhz": statistics.median(m for m, _ in got), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(got), "source": "NVML every %g ms" % (1e3 * self.period)}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -305,6 +398,23 @@ def cpu_baseline(cfg, target_s):
             "query_tokens_per_s": n_rows / t, "sample": _sample_text(cfg, n_rows, t)}
 
 
+def headline_config(cfg, B, world, args) -> dict:
+    """The `config` object of the headline line, computed from the shapes and arguments alone, so that
+    the GPU arm and the reference arm print the same one."""
+    rotate, fused = args.l2 == "rotate", args.path == "fused"
+    cache_mb = E2E_LAYERS * B * cfg.window_tokens * cfg.d_qk * 2 / 1e6
+    inputs_mb = N_INPUT_SETS * 2 * B * cfg.chunk_tokens * (cfg.dim + cfg.n_heads * (cfg.d_nope + cfg.d_rope)) / 1e6
+    return {"workload": "wan1.3b_layer_stream_step", "batch_per_gpu": B, "global_batch": B * world,
+            "query_tokens": cfg.chunk_tokens, "cached_tokens": cfg.window_tokens,
+            "heads": cfg.n_heads, "d_c": cfg.d_c, "d_rope": cfg.d_rope, "d_v": cfg.d_v,
+            "dim": cfg.dim, "parallelism": f"dp{world} (independent sequences)",
+            "l2": ("inputs larger than L2: steps cycle over %d layer caches (%.0f MB) and %d input sets (%.0f MB)"
+                   % (E2E_LAYERS, cache_mb, N_INPUT_SETS, inputs_mb) if rotate
+                   else "flushed between steps (512 MB write)"),
+            "path": ("compress + fused absorb/attention/value-up" if fused
+                     else "compress + absorb + attention + value-up")}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -325,8 +435,7 @@ def run_reference(args):
             "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "wan1.3b_layer_stream_step", "batch_per_gpu": 1,
-                       "query_tokens": cfg.chunk_tokens, "cached_tokens": cfg.window_tokens},
+            "config": headline_config(cfg, args.batch, args.gpus, args),
             "impl": "reference",
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": _sample_text(cfg, n_rows, t / args.steps) + " (per step)"},
@@ -731,19 +840,23 @@ def main():
     assert V.device_status() == 0
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local)          # 100 ms samples over the timed region and every leg after it
+    nvml = NvmlSampler(local)             # 2 ms samples: the timed region itself may last only ~20 ms
+    nvml.start()
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
     launches0 = V.launch_count()
+    nvml.mark("timed")
     wall0 = time.perf_counter()
     for i in range(args.steps):
         step(args.warmup + i, evs[i])
         between_steps()
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
+    nvml.mark("timed", end=True)
+    after_timed = clocks.snapshot()       # one blocking sample right after the timed region
     launches = V.launch_count() - launches0
-    clk = clocks.stop()
     barrier(world)
     per_kernel = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)] for j, n in enumerate(names)}
     step_ms = [evs[i][0].elapsed_time(evs[i][n_ev - 1]) for i in range(args.steps)]
@@ -827,6 +940,28 @@ def main():
                   "the first submit to the last output in host memory, max over ranks"}
     del e_caches
 
+    # ---- sustained: the same step back to back for at least a second (not part of `value`): a long
+    # run settles at the clock the 1 kW power cap allows, below the burst clock of a short one ----
+    sus_steps = int(min(20000, max(200, math.ceil(1.2e3 / statistics.mean(step_ms)))))
+    sus_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(sus_steps)]
+    torch.cuda.synchronize()
+    nvml.mark("sustained")
+    for i in range(sus_steps):
+        step(args.warmup + args.steps + 2 * ab_steps + i, sus_ev[i])
+        between_steps()
+    torch.cuda.synchronize()
+    nvml.mark("sustained", end=True)
+    sus_step = [sus_ev[i][0].elapsed_time(sus_ev[i][n_ev - 1]) for i in range(sus_steps)]
+    sus_k3 = statistics.mean(sus_ev[i][names.index(k3)].elapsed_time(sus_ev[i][names.index(k3) + 1])
+                             for i in range(sus_steps))
+    sustained = {"steps": sus_steps, "seconds": sum(sus_step) / 1e3, "ms_per_step": statistics.mean(sus_step),
+                 "tflops": f_step / (statistics.mean(sus_step) * 1e-3) / 1e12,
+                 "dominant_kernel_ms": sus_k3, "dominant_kernel_tflops": k3_flops / (sus_k3 * 1e-3) / 1e12,
+                 "frac_of_burst_peak": k3_flops / (sus_k3 * 1e-3) / 1e12 / pk["bf16_tflops"],
+                 "frac_of_sustained_peak": k3_flops / (sus_k3 * 1e-3) / 1e12 / pk["bf16_tflops_sustained"],
+                 "clocks": nvml.window("sustained")}
+    assert V.device_status() == 0
+
     # ---- dense per-head MHA comparison on the same shapes (not part of `value`) ----
     comparison = None
     if not args.no_dense:
@@ -870,6 +1005,14 @@ def main():
                       "cache_bytes_ratio": V.latent_cache_bytes(cfg, B) / V.dense_cache_bytes(cfg, B)}
         assert V.device_status() == 0
 
+    run_clocks = clocks.stop()
+    nvml.stop()
+    # the clocks line: the 2 ms NVML samples inside the timed region; the 100 ms nvidia-smi samples of
+    # the whole run and one blocking sample right after the timed region beside them
+    clk = nvml.window("timed") or (dict(after_timed, samples=1, source="nvidia-smi right after the timed region")
+                                   if after_timed else run_clocks)
+    if clk is not None:
+        clk = dict(clk, nvidia_smi_run=run_clocks, nvidia_smi_after_timed=after_timed)
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -878,22 +1021,12 @@ def main():
                 "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": "wan1.3b_layer_stream_step", "batch_per_gpu": B, "global_batch": B * world,
-                           "query_tokens": cfg.chunk_tokens, "cached_tokens": cfg.window_tokens,
-                           "heads": cfg.n_heads, "d_c": cfg.d_c, "d_rope": cfg.d_rope, "d_v": cfg.d_v,
-                           "dim": cfg.dim, "parallelism": f"dp{world} (independent sequences)",
-                           "l2": ("inputs larger than L2: steps cycle over %d layer caches (%.0f MB) and %d input "
-                                  "sets (%.0f MB)" % (len(caches), len(caches) * V.latent_cache_bytes(cfg, B) / 1e6,
-                                                      N_INPUT_SETS, N_INPUT_SETS * 2 * (xs[0].numel() + qs[0][0].numel() +
-                                                                                     qs[0][1].numel()) / 1e6)
-                                  if rotate else "flushed between steps (512 MB write)"),
-                           "path": ("compress + fused absorb/attention/value-up" if fused
-                                    else "compress + absorb + attention + value-up")},
+                "config": headline_config(cfg, B, world, args),
                 "query_tokens_per_s": q_tok_s,
                 "pct_of_bf16_peak": 100.0 * value / world / pk["bf16_tflops"],
                 "roofline": roofline, "kernels": kernels, "e2e": e2e, "gpu_launches": launches,
                 "clocks": clk, "wall_s_timed": wall, "cpu_baseline": cpu, "path_ab": path_ab,
-                "comparison": comparison}
+                "sustained": sustained, "comparison": comparison}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
