@@ -64,6 +64,8 @@ def parse():
                     help="fused: compress + one fused attention launch per step; three: compress + "
                          "absorb + attention + value-up launches (the other path is timed beside it)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sustained-seconds", type=float, default=1.2,
+                    help="length of the sustained leg (the step back to back; 0 leaves it out)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--workload", default="layer", choices=["layer", "batch8", "dc_sweep", "rollout", "fewstep",
                                                             "capacity"],
@@ -942,7 +944,8 @@ def main():
 
     # ---- sustained: the same step back to back for at least a second (not part of `value`): a long
     # run settles at the clock the 1 kW power cap allows, below the burst clock of a short one ----
-    sus_steps = int(min(20000, max(200, math.ceil(1.2e3 / statistics.mean(step_ms)))))
+    sus_steps = (int(min(20000, max(200, math.ceil(args.sustained_seconds * 1e3 / statistics.mean(step_ms)))))
+                 if args.sustained_seconds > 0 else 0)
     sus_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(sus_steps)]
     torch.cuda.synchronize()
     nvml.mark("sustained")
@@ -951,10 +954,10 @@ def main():
         between_steps()
     torch.cuda.synchronize()
     nvml.mark("sustained", end=True)
-    sus_step = [sus_ev[i][0].elapsed_time(sus_ev[i][n_ev - 1]) for i in range(sus_steps)]
-    sus_k3 = statistics.mean(sus_ev[i][names.index(k3)].elapsed_time(sus_ev[i][names.index(k3) + 1])
-                             for i in range(sus_steps))
-    sustained = {"steps": sus_steps, "seconds": sum(sus_step) / 1e3, "ms_per_step": statistics.mean(sus_step),
+    sus_step = [sus_ev[i][0].elapsed_time(sus_ev[i][n_ev - 1]) for i in range(sus_steps)] or [float("nan")]
+    sus_k3 = statistics.mean([sus_ev[i][names.index(k3)].elapsed_time(sus_ev[i][names.index(k3) + 1])
+                              for i in range(sus_steps)] or [float("nan")])
+    sustained = None if not sus_steps else {"steps": sus_steps, "seconds": sum(sus_step) / 1e3, "ms_per_step": statistics.mean(sus_step),
                  "tflops": f_step / (statistics.mean(sus_step) * 1e-3) / 1e12,
                  "dominant_kernel_ms": sus_k3, "dominant_kernel_tflops": k3_flops / (sus_k3 * 1e-3) / 1e12,
                  "frac_of_burst_peak": k3_flops / (sus_k3 * 1e-3) / 1e12 / pk["bf16_tflops"],

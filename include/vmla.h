@@ -175,7 +175,7 @@ VMLA_API vmla_status vmla_latent_attention(const vmla_config* cfg, const void* q
  *   q_nope [batch, Nq, n_heads, d_nope], q_rope [batch, Nq, n_heads, d_rope],
  *   w_uk [n_heads, d_nope, d_c], w_uv [n_heads, d_v, d_c]
  *   -> out [batch, Nq, n_heads, d_v], lse [batch, Nq, n_heads] (natural log, or NULL).
- * Same window rules as vmla_latent_attention.  bf16 only; needs d_rope == 32, d_c in {128, 192, 256},
+ * Same window rules as vmla_latent_attention.  bf16 only; needs d_rope == 32, d_c in {64, 128, 192, 256},
  * d_nope a multiple of 16 in [16, 128] and d_v a multiple of 32 in [32, 128] (VMLA_ERR_UNSUPPORTED
  * otherwise). */
 VMLA_API vmla_status vmla_latent_attention_fused(const vmla_config* cfg, const void* q_nope, const void* q_rope,
@@ -330,7 +330,7 @@ VMLA_API int32_t vmla_debug_shrink_extents(int64_t bytes);
  * iteration), n added to the exponent field; arguments below -125 are clamped to -125.  Claimed
  * accuracy: relative error <= 7.5e-5 for -125 <= x <= 120, and 2^-125 within that error for x < -125,
  * -inf and NaN.  y[i] = that 2^x of x[i], i < n: x and y are device buffers of n floats; the kernel
- * runs on `stream`.  VMLA_ERR_INVALID_ARG on NULL pointers or n < 0. */
+ * runs on `stream`.  n == 0 does nothing; VMLA_ERR_INVALID_ARG on n < 0 or NULL pointers with n > 0. */
 VMLA_API vmla_status vmla_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream);
 
 /* Number of kernels the library has launched in this process (all entry points, all devices). */

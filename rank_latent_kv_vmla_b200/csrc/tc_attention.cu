@@ -118,7 +118,10 @@ struct Plan {
   static constexpr int kNPV = kDV + (ONES ? 16 : 0);     // N of the P V MMA
   static constexpr int kBox = BN * 128;                 // [BN x 64] bf16 box, 128-byte swizzle
   static constexpr int kRopeBox = BN * 64;              // [BN x 32] bf16 box, 64-byte swizzle
-  static constexpr int kQBytes = Q_TMEM ? 0 : (KB * kBlockM * 128 + (KR ? kBlockM * 64 : 0));
+  // Q buffer: the c boxes, then the rope box; the fused prologue first stages q^nope (two boxes) there
+  static constexpr int kQBoxes = (FUSED && KB < 2) ? 2 : KB;
+  static constexpr int kQRopeOff = kQBoxes * kBlockM * 128;
+  static constexpr int kQBytes = Q_TMEM ? 0 : (kQRopeOff + (KR ? kBlockM * 64 : 0));
   // stage layout: c boxes (K, and V = the first VB of them) | ones box | rope box
   static constexpr int kOnesOff = KB * kBox;
   static constexpr int kRopeOff = kOnesOff + (ONES ? kBox : 0);
@@ -140,8 +143,8 @@ struct Plan {
   static_assert(!ONES || Q_TMEM, "the ones box is filled by the warps that also write Q into TMEM");
   static_assert(kNPV <= 256 && kNPV % 16 == 0, "P V MMA shape");
   // fused: q^nope (two 64-column boxes) and then O / l must fit the Q buffer
-  static_assert(!FUSED || (!Q_TMEM && KR == 32 && !ONES && KB >= 2 &&
-                           kQBytes >= 2 * kBlockM * 128 && kQBytes >= VB * kBlockM * 128),
+  static_assert(!FUSED || (!Q_TMEM && KR == 32 && !ONES &&
+                           kQRopeOff >= 2 * kBlockM * 128 && kQRopeOff >= VB * kBlockM * 128),
                 "fused layout");
 };
 
@@ -224,7 +227,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       if (!Q_TMEM && !FUSED) {
         mbar_arrive_expect_tx(bar_q, PL::kQBytes);
         for (int i = 0; i < KB; ++i) tma_load_4d(sQ + i * kBlockM * 128, &map_q, bar_q, 64 * i, h, row0, b);
-        if (KR) tma_load_4d(sQ + KB * kBlockM * 128, &map_qr, bar_q, 64 * KB, h, row0, b);
+        if (KR) tma_load_4d(sQ + PL::kQRopeOff, &map_qr, bar_q, 64 * KB, h, row0, b);
       }
       if (FUSED) {
         // prologue operands: the q^nope tile (two 64-column boxes; columns past d_nope read as zeros)
@@ -346,7 +349,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             if (Q_TMEM) {
               mma_ts(s_addr, tmem + PL::kTmemQ + KB * 32 + k * 8, kdesc, idesc_qk, 1u);
             } else {
-              const uint64_t qdesc = smem_desc(q_base + KB * kBlockM * 128 + k * 32, 16, 512, kSwizzle64B);
+              const uint64_t qdesc = smem_desc(q_base + PL::kQRopeOff + k * 32, 16, 512, kSwizzle64B);
               mma_ss(s_addr, qdesc, kdesc, idesc_qk, 1u);
             }
           }
@@ -458,7 +461,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           v[2 * q] = a;
           v[2 * q + 1] = bb;
         }
-        uint8_t* ropep = sQ + KB * (kBlockM * 128) + r * 64;
+        uint8_t* ropep = sQ + PL::kQRopeOff + r * 64;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint4 w;
@@ -777,8 +780,8 @@ bool fused_fits(int d_nope, int d_v) {
 
 vmla_status tc_check_fused_attention(const vmla_config& c) {
   if (c.d_rope != 32) { set_tc_reason("fused latent attention needs d_rope == 32"); return VMLA_ERR_UNSUPPORTED; }
-  if (c.d_c != 128 && c.d_c != 192 && c.d_c != 256) {
-    set_tc_reason("fused latent attention needs d_c in {128, 192, 256}");
+  if (c.d_c != 64 && c.d_c != 128 && c.d_c != 192 && c.d_c != 256) {
+    set_tc_reason("fused latent attention needs d_c in {64, 128, 192, 256}");
     return VMLA_ERR_UNSUPPORTED;
   }
   if (c.d_nope % 16 || c.d_nope < 16 || c.d_nope > 128) {
@@ -789,7 +792,8 @@ vmla_status tc_check_fused_attention(const vmla_config& c) {
     set_tc_reason("fused latent attention needs d_v a multiple of 32 in [32, 128]");
     return VMLA_ERR_UNSUPPORTED;
   }
-  const bool fits = c.d_c == 128 ? fused_fits<2>(c.d_nope, c.d_v)
+  const bool fits = c.d_c == 64 ? fused_fits<1>(c.d_nope, c.d_v)
+                    : c.d_c == 128 ? fused_fits<2>(c.d_nope, c.d_v)
                     : c.d_c == 192 ? fused_fits<3>(c.d_nope, c.d_v) : fused_fits<4>(c.d_nope, c.d_v);
   if (!fits) { set_tc_reason("fused latent attention: up-projection weights exceed a KV stage"); return VMLA_ERR_UNSUPPORTED; }
   return VMLA_OK;
@@ -840,6 +844,7 @@ cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t
   p.lse_span = make_span(lse, checked_extent((int64_t)batch * nq * H * 4));
   const int n_tiles = batch * H * p.tiles_per_group;
   switch (dc) {
+    case 64: return launch_attention<1, 32, 1, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
     case 128: return launch_attention<2, 32, 2, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
     case 192: return launch_attention<3, 32, 3, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);
     default: return launch_attention<4, 32, 4, kLatentBN, 2, false, false, true>(m, p, n_tiles, st);

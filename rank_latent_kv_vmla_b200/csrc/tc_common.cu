@@ -111,8 +111,9 @@ __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict_
 }  // namespace vmla
 
 extern "C" VMLA_API vmla_status vmla_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
-  if (!x || !y || n < 0) return vmla::report(VMLA_ERR_INVALID_ARG, "x and y must not be NULL and n >= 0");
-  if (n == 0) return VMLA_OK;
+  if (n < 0) return vmla::report(VMLA_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return VMLA_OK;                       // nothing to do (empty buffers may be NULL)
+  if (!x || !y) return vmla::report(VMLA_ERR_INVALID_ARG, "x and y must not be NULL");
   const int64_t pairs = (n + 1) / 2;
   const int threads = 256;
   const int64_t want = (pairs + threads - 1) / threads;

@@ -175,7 +175,7 @@ def test_plan_capacity_rejects_bad_arguments():
 def test_fused_attention_rejects_unsupported_shapes():
     """The fused call refuses, before launching, the fp32 path and shapes outside its layout."""
     cache = _cache(frames_written=TINY.chunk_frames)
-    for bad, why in ((TINY, "bf16"), (WAN.replace(d_c=64), "d_c"), (WAN.replace(d_nope=88, rope_pairs_t=6), "d_nope"),
+    for bad, why in ((TINY, "bf16"), (WAN.replace(d_c=96), "d_c"), (WAN.replace(d_nope=88, rope_pairs_t=6), "d_nope"),
                      (WAN.replace(d_v=160), "d_v")):
         cc = V.c_config(bad)
         c = _cache(frames_written=bad.chunk_frames)
@@ -275,7 +275,8 @@ def test_cache_checkpoint_round_trip(tmp_path):
     (WAN, True),
     (WAN.replace(d_c=128), True),
     (WAN.replace(d_c=256), True),
-    (WAN.replace(d_c=64), False),        # the fused kernel needs d_c in {128, 192, 256}
+    (WAN.replace(d_c=64), True),
+    (WAN.replace(d_c=96), False),        # the fused kernel needs d_c in {64, 128, 192, 256}
     (WAN.replace(d_nope=104, rope_pairs_t=6), False),   # d_nope not a multiple of 16
     (TINY, False),                       # fp32 runs on the SIMT path only
 ])

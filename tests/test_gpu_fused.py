@@ -73,9 +73,15 @@ def test_mid_fused_streaming_multitile(V):
     _stream_fused(V, MID.replace(grid_h=12, grid_w=12), batch=2, n_steps=4, seed=3050)
 
 
-@pytest.mark.parametrize("d_c", [128, 256])
+@pytest.mark.parametrize("d_c", [64, 128, 256])
 def test_mid_fused_latent_sizes(V, d_c):
     _stream_fused(V, MID.replace(d_c=d_c), batch=1, n_steps=3, seed=3100 + d_c)
+
+
+def test_mid_fused_lowest_rank_multitile(V):
+    """d_c = 64 (one latent box; q^nope still staged in two boxes) with 288-token chunks, B = 2, the
+    ring wrapping."""
+    _stream_fused(V, MID.replace(d_c=64, grid_h=12, grid_w=12), batch=2, n_steps=4, seed=3150)
 
 
 def test_mid_fused_narrow_heads(V):

@@ -231,7 +231,7 @@ def test_tiny_fp32_dense_path(V):
     assert_close(f64(o_d[0]), ref["o"], cfg, "dense o")
 
 
-@pytest.mark.parametrize("batch", [1, 2])
+@pytest.mark.parametrize("batch", [1, 2, 4])
 def test_wan_full_size_sampled(V, batch):
     """The Wan-1.3B-shaped layer at full size: 8 chunks streamed into the 21-frame window (the last
     one evicts frames 0-2); whole cache planes and all absorbed queries are checked, attention and
