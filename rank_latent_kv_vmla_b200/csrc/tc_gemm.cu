@@ -1,5 +1,9 @@
 // Projection GEMMs of the VideoMLA path on the sm_100a tensor cores (tcgen05 + TMEM + TMA), each
-// with its own fused epilogue (the compress + ring append has its own kernel, tc_compress.cu):
+// with its own fused epilogue:
+//   compress_append  [c ; W^KR x] = [W^KV_down ; W^KR] x, 3D-RoPE on the last d_rope columns, bf16
+//                    store into the ring rows of the chunk's frames (Method items 1 and 3); also a
+//                    token range of the chunk into several replicas of the ring (peer mappings), and
+//                    the column tile narrows to 128 / 64 when the row tiles alone leave SMs idle;
 //   absorb_q         q~_h = (W^K_up,h)^T q^nope_h per head (B operand read MN-major from W^K_up as
 //                    stored), plus RoPE3D(q^rope_h) written beside it (Method items 2 and 3);
 //   value_up         o_h = W^V_up,h o~_h per head (Method item 2);
@@ -18,7 +22,6 @@
 #include "ptx_sm100.cuh"
 #include "tc_common.cuh"
 #include "tc_kernels.cuh"
-#include "tc_proj_common.cuh"
 
 namespace vmla {
 namespace {
@@ -54,7 +57,104 @@ __device__ __forceinline__ void store32(bf16* dst, const float* v) {
   }
 }
 
+// 3D-RoPE of the epilogues through a per-CTA table: cos/sin of every (rotary pair, position along its
+// axis) that the call can meet -- the call's frames, every row, every column -- computed once per CTA
+// in shared memory (angle reduced in double precision, then sincosf).  Pair p's entries start at
+// off[p]; frame positions are stored relative to base_f.  n_entries == 0 (table too large) falls back
+// to computing each rotation directly.
+constexpr int kRopeTabEntries = 2048;
+
+struct RopeLookup {
+  RopeTable rt;
+  int off[kMaxRopePairs];
+  int64_t base_f;
+  int n_entries;
+  __device__ void rotate32(const float2* tab, int pair0, int64_t f, int64_t i, int64_t j, float* v) const {
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int p = pair0 + q;
+      float a, b;
+      if (n_entries) {
+        const int ax = rt.axis[p];
+        const int64_t pos = ax == 0 ? f - base_f : (ax == 1 ? i : j);
+        const float2 cs = tab[off[p] + pos];
+        a = v[2 * q] * cs.x - v[2 * q + 1] * cs.y;
+        b = v[2 * q] * cs.y + v[2 * q + 1] * cs.x;
+      } else {
+        rope_rotate_f32(rt, p, f, i, j, v[2 * q], v[2 * q + 1], &a, &b);
+      }
+      v[2 * q] = a;
+      v[2 * q + 1] = b;
+    }
+  }
+
+  // fill the table with threads t0 .. t0 + nthreads - 1 (the caller synchronises them afterwards).  The
+  // angle is reduced to [-pi, pi] in double precision, then the MUFU sine / cosine (absolute error
+  // about 1e-6 there, far below the bf16 rounding of the rotated values) keep the build short.
+  __device__ void build(float2* smem_tab, int t0, int nthreads) const {
+    const double two_pi = 6.283185307179586476925286766559;
+    const double inv_two_pi = 0.15915494309189533576888376337251;
+    for (int e = t0; e < n_entries; e += nthreads) {
+      int p = 0;
+      while (p + 1 < rt.n_pairs && off[p + 1] <= e) ++p;
+      const int64_t v = e - off[p];
+      const double pos = (double)(rt.axis[p] == 0 ? base_f + v : v);
+      double ang = pos * rt.inv_freq[p];
+      ang = fma(-two_pi, rint(ang * inv_two_pi), ang);
+      float sn, cs;
+      __sincosf((float)ang, &sn, &cs);
+      smem_tab[e] = make_float2(cs, sn);
+    }
+  }
+};
+
+// Host: table layout for a call whose tokens span `frames` frames starting at g.first_frame.
+RopeLookup make_rope_lookup(const RopeTable& rt, const FrameGeom& g, int frames) {
+  RopeLookup L{};
+  L.rt = rt;
+  L.base_f = g.first_frame;
+  const int extent[3] = {frames, g.tokens_per_frame / g.grid_w, g.grid_w};
+  int total = 0;
+  for (int p = 0; p < rt.n_pairs; ++p) {
+    L.off[p] = total;
+    total += extent[rt.axis[p]];
+  }
+  L.n_entries = total <= kRopeTabEntries ? total : 0;
+  return L;
+}
+
 // ---- epilogues: called per (row m, 32-column chunk starting at col0) with the fp32 values ----
+// Row m of the GEMM is token tok0 + m % ntok of batch element m / ntok; its c and k^R rows go to the
+// ring of every destination cache (several when replicas of the cache live on other GPUs: plain stores
+// through peer mappings, so the exchange of the chunk's latents is done by this epilogue).
+struct EpiCompress {
+  static constexpr bool kRope = true;
+  bf16* c[kMaxCacheDst]; bf16* k_r[kMaxCacheDst]; int n_dst;
+  int d_c, d_rope; int64_t ntok, tok0, cap; FrameGeom g; RopeLookup rope;
+  Span c_span[kMaxCacheDst], kr_span[kMaxCacheDst]; int* status;
+  __device__ void operator()(const float2* tab, int, int64_t m, int col0, float* v) const {
+    const int64_t b = m / ntok, tok = tok0 + m % ntok;
+    const int64_t row = b * cap + ring_row(g, tok);
+    if (col0 < d_c) {
+      for (int d = 0; d < n_dst; ++d) {
+        bf16* q = c[d] + row * d_c + col0;
+        if (store_ok(c_span[d], q, 64, status, 1)) store32(q, v);
+      }
+    } else {
+      const int64_t f = g.first_frame + tok / g.tokens_per_frame;
+      const int64_t r = tok % g.tokens_per_frame;
+      rope.rotate32(tab, (col0 - d_c) / 2, f, r / g.grid_w, r % g.grid_w, v);
+      for (int d = 0; d < n_dst; ++d) {
+        bf16* q = k_r[d] + row * d_rope + (col0 - d_c);
+        if (store_ok(kr_span[d], q, 64, status, 2)) store32(q, v);
+      }
+    }
+    // stores to other GPUs' memory: make them visible system-wide before this thread goes on
+    if (n_dst > 1) __threadfence_system();
+  }
+  __device__ void finish(const float2*, int, int64_t) const {}
+};
+
 struct EpiAbsorb {
   static constexpr bool kRope = true;
   bf16* q_abs; const bf16* q_rope; int heads, d_c, d_rope; int64_t nq; FrameGeom g; RopeLookup rope;
@@ -306,6 +406,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ C
   }
 }
 
+int num_sms() {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cached[dev] = v;
+  }
+  return cached[dev];
+}
+
 // One CTA per SM (TMEM holds two accumulators), each looping over its share of the tiles.
 template <int BN, bool B_MN_MAJOR, class Epi>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmShape& sh, int heads,
@@ -326,7 +438,16 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmSh
 
 }  // namespace
 
+static int pick_bn(int N);
 static bool bn_supported(int bn, bool mn_major);
+
+vmla_status tc_check_compress(const vmla_config& c) {
+  if (c.d_rope != 32 || c.d_c % 32 || c.dim % 8 || !bn_supported(pick_bn(c.d_c + c.d_rope), false)) {
+    set_tc_reason("tensor-core compress needs d_rope == 32, d_c % 32 == 0, dim % 8 == 0");
+    return VMLA_ERR_UNSUPPORTED;
+  }
+  return VMLA_OK;
+}
 
 vmla_status tc_check_absorb(const vmla_config& c) {
   if (c.d_rope % 32 || !bn_supported(c.d_c, true) || c.d_nope % 8) {
@@ -354,6 +475,10 @@ vmla_status tc_check_dense_append(const vmla_config& c) {
   return VMLA_OK;
 }
 
+// Column tile used for an N-wide projection: the whole N when it fits one tcgen05.mma (N <= 256),
+// else 160-column tiles.  Every candidate is a multiple of 32 (epilogue chunks) and of 16 (MMA N).
+static int pick_bn(int N) { return N <= 256 ? N : 160; }
+
 template <bool B_MN_MAJOR, class Epi>
 static cudaError_t dispatch_bn(int bn, const CUtensorMap& a, const CUtensorMap& b, const GemmShape& sh,
                                int heads, const Epi& epi, cudaStream_t st) {
@@ -378,6 +503,55 @@ static cudaError_t dispatch_bn(int bn, const CUtensorMap& a, const CUtensorMap& 
 static bool bn_supported(int bn, bool mn_major) {
   if (bn == 64 || bn == 128 || bn == 192 || bn == 256) return true;
   return !mn_major && (bn == 96 || bn == 160 || bn == 224);
+}
+
+cudaError_t tc_compress_append(const vmla_config& cfg, int batch, const void* x, const void* w,
+                               const FrameGeom& g, const RopeTable& rt, void* c, void* k_r,
+                               cudaStream_t st) {
+  CacheDst d{c, k_r};
+  return tc_compress_rows(cfg, batch, 0, (int64_t)cfg.chunk_frames * cfg.grid_h * cfg.grid_w, x, w, g, rt,
+                          &d, 1, st);
+}
+
+cudaError_t tc_compress_rows(const vmla_config& cfg, int batch, int64_t tok0, int64_t ntok, const void* x,
+                             const void* w, const FrameGeom& g, const RopeTable& rt, const CacheDst* dst,
+                             int n_dst, cudaStream_t st) {
+  if (n_dst < 1 || n_dst > kMaxCacheDst) return cudaErrorInvalidValue;
+  const int64_t M = batch * ntok;
+  const int N = cfg.d_c + cfg.d_rope, K = cfg.dim;
+  // one 224-wide column tile per 128 rows leaves most SMs idle at small batch: narrow the column tile
+  // until the tiles cover the SMs (the x tile is then re-read from L2 by each column tile; the RoPE
+  // columns d_c .. d_c+31 stay inside one 32-column chunk of one tile because d_c % 32 == 0)
+  int bn = pick_bn(N);
+  const int64_t m_tiles = (M + kBM - 1) / kBM;
+  for (int cand : {128, 64})
+    if (m_tiles * ((N + bn - 1) / bn) < num_sms() && cand < bn) bn = cand;
+  CUtensorMap ma, mb;
+  cudaError_t e;
+  // A = x [M, D]; B = [W^KV_down ; W^KR] [N, D], both K-major
+  if ((e = make_map_4d(&ma, x, K, 1, M, 1, (int64_t)K * 2, (int64_t)K * 2, M * K * 2, kBK, 1, kBM, 128)) != cudaSuccess)
+    return e;
+  if ((e = make_map_4d(&mb, w, K, N, 1, 1, (int64_t)K * 2, (int64_t)N * K * 2, (int64_t)N * K * 2, kBK, bn, 1, 128)) != cudaSuccess)
+    return e;
+  GemmShape sh{M, N, K, 0, wait_limit_ns(), device_status_ptr()};
+  EpiCompress epi{};
+  const int64_t cap_rows = (int64_t)batch * cfg.window_frames * cfg.grid_h * cfg.grid_w;
+  for (int d = 0; d < n_dst; ++d) {
+    epi.c[d] = (bf16*)dst[d].c;
+    epi.k_r[d] = (bf16*)dst[d].k_r;
+    epi.c_span[d] = make_span(dst[d].c, checked_extent(cap_rows * cfg.d_c * 2));
+    epi.kr_span[d] = make_span(dst[d].k_r, checked_extent(cap_rows * cfg.d_rope * 2));
+  }
+  epi.status = device_status_ptr();
+  epi.n_dst = n_dst;
+  epi.d_c = cfg.d_c;
+  epi.d_rope = cfg.d_rope;
+  epi.ntok = ntok;
+  epi.tok0 = tok0;
+  epi.cap = (int64_t)cfg.window_frames * cfg.grid_h * cfg.grid_w;
+  epi.g = g;
+  epi.rope = make_rope_lookup(rt, g, cfg.chunk_frames);
+  return dispatch_bn<false>(bn, ma, mb, sh, 1, epi, st);
 }
 
 cudaError_t tc_absorb_q(const vmla_config& cfg, int batch, int64_t nq, const void* q_nope,
