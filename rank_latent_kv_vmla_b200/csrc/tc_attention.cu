@@ -62,24 +62,6 @@ constexpr int kPolyPairs = VMLA_EXP2_POLY_PAIRS;
 #endif
 constexpr int kPParts = VMLA_P_PARTS;
 
-// Rotation of query pair p for the fused prologue: the angle is formed and reduced to [-pi, pi] in
-// double precision (large frame indices lose nothing), then the MUFU sine / cosine (absolute error
-// about 1e-6 on that interval, far below the bf16 rounding of the result) keep this once-per-row
-// step short.
-__device__ __forceinline__ void rope_rotate_mufu(const RopeTable& rt, int p, int64_t f, int64_t i, int64_t j,
-                                                 float a, float b, float* ra, float* rb) {
-  const int ax = rt.axis[p];
-  const double pos = (double)(ax == 0 ? f : (ax == 1 ? i : j));
-  const double two_pi = 6.283185307179586476925286766559;
-  const double inv_two_pi = 0.15915494309189533576888376337251;
-  double ang = pos * rt.inv_freq[p];
-  ang = fma(-two_pi, rint(ang * inv_two_pi), ang);
-  float sf, cf;
-  __sincosf((float)ang, &sf, &cf);
-  *ra = a * cf - b * sf;
-  *rb = a * sf + b * cf;
-}
-
 struct AttnParams {
   const void* q;         // query rows (used when Q is kept in TMEM)
   int rows_per_b;        // query rows per batch element (token-major: Nq*H, head-major: Nq)
@@ -724,6 +706,9 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
                                 const void* c, const void* k_r, int64_t cap, int64_t valid_rows,
                                 const FrameGeom& g, float scale, void* out, float* lse, int* status,
                                 cudaStream_t st) {
+  // d_c = 64 / 128: the softmax chain, not the tensor cores, bounds a single softmax warpgroup there
+  if (tc_latent_split_supported(cfg))
+    return tc_latent_attention_split(cfg, batch, nq, q_abs, c, k_r, cap, valid_rows, g, scale, out, lse, status, st);
   const int H = cfg.n_heads, dqk = cfg.d_c + cfg.d_rope;
   const int64_t rows = nq * H;
   const int kv_box_rows = kLatentBN;
@@ -758,8 +743,6 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
   p.lse_span = make_span(lse, checked_extent((int64_t)batch * rows * 4));
   const int n_tiles = batch * p.tiles_per_group;
   switch (cfg.d_c) {
-    case 64: return launch_attention<1, 32, 1, kLatentBN, 2, true, false, false>(m, p, n_tiles, st);
-    case 128: return launch_attention<2, 32, 2, kLatentBN, 2, true, false, false>(m, p, n_tiles, st);
     case 192: return launch_attention<3, 32, 3, kLatentBN, 2, false, false, false>(m, p, n_tiles, st);
     default: return launch_attention<4, 32, 4, kLatentBN, 2, false, false, false>(m, p, n_tiles, st);
   }
@@ -804,6 +787,10 @@ cudaError_t tc_latent_attention_fused(const vmla_config& cfg, int batch, int64_t
                                       const void* c, const void* k_r, int64_t cap, int64_t valid_rows,
                                       const FrameGeom& g, const RopeTable& rt, float scale, void* out, float* lse,
                                       int* status, cudaStream_t st) {
+  // d_c = 64 / 128: the softmax chain bounds a single softmax warpgroup; split each tile's keys
+  if (tc_latent_split_fused_supported(cfg))
+    return tc_latent_attention_split_fused(cfg, batch, tok0, nq, q_nope, q_rope, w_uk, w_uv, c, k_r, cap,
+                                           valid_rows, g, rt, scale, out, lse, status, st);
   const int H = cfg.n_heads, dn = cfg.d_nope, dc = cfg.d_c, dv = cfg.d_v;
   AttnMaps m{};
   cudaError_t e;

@@ -36,6 +36,21 @@ cudaError_t tc_latent_attention(const vmla_config& cfg, int batch, int64_t nq, c
                                 const FrameGeom& g, float scale, void* out, float* lse, int* status,
                                 cudaStream_t st);
 
+// The same call at d_c = 64 / 128, with the keys of every tile split between two softmax warpgroups.
+bool tc_latent_split_supported(const vmla_config& cfg);
+cudaError_t tc_latent_attention_split(const vmla_config& cfg, int batch, int64_t nq, const void* q_abs,
+                                      const void* c, const void* k_r, int64_t cap, int64_t valid_rows,
+                                      const FrameGeom& g, float scale, void* out, float* lse, int* status,
+                                      cudaStream_t st);
+
+// The fused call (below) at d_c = 64 / 128 with d_v a multiple of 64, keys split the same way.
+bool tc_latent_split_fused_supported(const vmla_config& cfg);
+cudaError_t tc_latent_attention_split_fused(const vmla_config& cfg, int batch, int64_t tok0, int64_t nq,
+                                            const void* q_nope, const void* q_rope, const void* w_uk,
+                                            const void* w_uv, const void* c, const void* k_r, int64_t cap,
+                                            int64_t valid_rows, const FrameGeom& g, const RopeTable& rt,
+                                            float scale, void* out, float* lse, int* status, cudaStream_t st);
+
 // Absorbed query, latent attention and value up-projection in one kernel (q_abs and the latent
 // output stay on chip): q_nope [B, Nq, H, d_nope], q_rope [B, Nq, H, 32] -> out [B, Nq, H, d_v].
 vmla_status tc_check_fused_attention(const vmla_config& cfg);

@@ -82,6 +82,24 @@ __device__ __forceinline__ void rope_rotate_f32(const RopeTable& rt, int p, int6
   *rb = a * sf + b * cf;
 }
 
+// Rotation of query pair p for the fused prologue: the angle is formed and reduced to [-pi, pi] in
+// double precision (large frame indices lose nothing), then the MUFU sine / cosine (absolute error
+// about 1e-6 on that interval, far below the bf16 rounding of the result) keep this once-per-row
+// step short.
+__device__ __forceinline__ void rope_rotate_mufu(const RopeTable& rt, int p, int64_t f, int64_t i, int64_t j,
+                                                 float a, float b, float* ra, float* rb) {
+  const int ax = rt.axis[p];
+  const double pos = (double)(ax == 0 ? f : (ax == 1 ? i : j));
+  const double two_pi = 6.283185307179586476925286766559;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
+  double ang = pos * rt.inv_freq[p];
+  ang = fma(-two_pi, rint(ang * inv_two_pi), ang);
+  float sf, cf;
+  __sincosf((float)ang, &sf, &cf);
+  *ra = a * cf - b * sf;
+  *rb = a * sf + b * cf;
+}
+
 // Device status word (bounded waits that ran out record a nonzero code here).
 int* device_status_ptr();   // address of this device's status word (host side), nullptr on error
 void count_launches(int n);

@@ -80,16 +80,20 @@ def _run(V, cfg, batch, n_chunks, seed, first_frame=0, check_from=0, fused=None)
                 assert_close(f64(o_f[b]), ref["o"], cfg, f"chunk {k} fused o b{b}")
 
 
-def test_window_of_one_chunk(V):
-    _run(V, MID.replace(window_frames=MID.chunk_frames), batch=2, n_chunks=3, seed=61)
+@pytest.mark.parametrize("d_c", [192, 64])
+def test_window_of_one_chunk(V, d_c):
+    _run(V, MID.replace(window_frames=MID.chunk_frames, d_c=d_c), batch=2, n_chunks=3, seed=61)
 
 
 def test_window_of_one_chunk_fp32(V):
     _run(V, TINY.replace(window_frames=1), batch=2, n_chunks=3, seed=62)
 
 
-def test_one_token_frames(V):
-    cfg = MID.replace(grid_h=1, grid_w=1, chunk_frames=1, window_frames=3)
+@pytest.mark.parametrize("d_c", [192, 64, 128])
+def test_one_token_frames(V, d_c):
+    """Three visible keys at most: at d_c = 64 / 128 the second key half of every tile is fully
+    masked (that warpgroup keeps m = -inf and contributes nothing to the merge)."""
+    cfg = MID.replace(grid_h=1, grid_w=1, chunk_frames=1, window_frames=3, d_c=d_c)
     _run(V, cfg, batch=3, n_chunks=5, seed=63)
 
 

@@ -79,11 +79,12 @@ def test_mid_bf16_streaming_every_call(V, batch):
     _stream_and_check(V, MID, batch=batch, n_steps=4, seed=2024 + batch)
 
 
-def test_mid_bf16_peaked_softmax_isolated(V):
+@pytest.mark.parametrize("d_c", [192, 64])
+def test_mid_bf16_peaked_softmax_isolated(V, d_c):
     """Queries x8 (peaked attention, exercises the running-max rescale).  Each call is fed the
     oracle's own bf16-rounded inputs, so only that call's arithmetic is measured: through the whole
     chain the x8 logits would amplify the bf16 storage rounding of q_abs and c beyond the tolerance."""
-    _isolated_attention_and_value_up(V, MID, seed=31, q_gain=8.0)
+    _isolated_attention_and_value_up(V, MID.replace(d_c=d_c), seed=31, q_gain=8.0)
 
 
 def _isolated_attention_and_value_up(V, cfg, seed, q_gain=1.0, batch=2, n_chunks=4):
@@ -133,7 +134,7 @@ def test_mid_bf16_attention_isolated(V):
     _isolated_attention_and_value_up(V, MID, seed=99)
 
 
-@pytest.mark.parametrize("d_c", [64, 256])
+@pytest.mark.parametrize("d_c", [64, 128, 256])
 def test_mid_bf16_attention_isolated_latent_sizes(V, d_c):
     _isolated_attention_and_value_up(V, MID.replace(d_c=d_c), seed=98 + d_c, batch=1)
 
@@ -276,10 +277,12 @@ def test_native_kernels_launched(V):
     assert V.launch_count() > before
 
 
-def test_bounded_wait_reports_timeout_and_context_survives(V):
+@pytest.mark.parametrize("d_c", [192, 64])
+def test_bounded_wait_reports_timeout_and_context_survives(V, d_c):
     """A KV tile that is never loaded makes the consumer's bounded wait run out: the kernel returns,
-    vmla_device_status reports a nonzero code, and the next call on the same context is correct."""
-    cfg = MID
+    vmla_device_status reports a nonzero code, and the next call on the same context is correct
+    (d_c = 64 runs the kernel whose tile keys are split between two softmax warpgroups)."""
+    cfg = MID.replace(d_c=d_c)
     inp = synthetic.draw_layer(cfg, batch=1, seed=404, n_chunks=3)
     cache = V.LatentCache(cfg, 1, device=DEV)
     for x in inp.x_chunks:

@@ -10,7 +10,7 @@ import torch
 from oracle import vmla_oracle as O
 from rank_latent_kv_vmla_b200.config import WAN
 import synthetic
-from parity import OracleLayer, assert_close, dense_weights_from_latent, errors, f64, round_to, pairs
+from parity import OracleLayer, assert_close, dense_weights_from_latent, errors, f64, round_to, pairs, paths_rel_tol
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -59,7 +59,7 @@ def test_wan_batch8_latent_and_dense_agree_with_oracle(V):
     for b in range(B):
         assert_close(f64(o_d[b]), f64(o_l[b]), cfg, f"dense vs latent b{b}")
         rel_l2, max_ratio = errors(f64(o_f[b]), f64(o_l[b]))
-        assert rel_l2 <= 2e-3 and max_ratio <= 1e-2, (b, rel_l2, max_ratio)
+        assert rel_l2 <= paths_rel_tol(cfg) and max_ratio <= 1e-2, (b, rel_l2, max_ratio)
     # and sampled rows of the first and last sequence against the oracle
     orc = OracleLayer(cfg, inp, B)
     rows = _rows(cfg)
@@ -99,7 +99,7 @@ def test_wan_lower_rank_batch16(V, d_c):
     assert cache.nbytes() == V.latent_cache_bytes(cfg, B)
     for b in range(B if fused else 0):
         rel_l2, max_ratio = errors(f64(o_f[b]), f64(o[b]))
-        assert rel_l2 <= 2e-3 and max_ratio <= 1e-2, (b, rel_l2, max_ratio)
+        assert rel_l2 <= paths_rel_tol(cfg) and max_ratio <= 1e-2, (b, rel_l2, max_ratio)
     orc = OracleLayer(cfg, inp, B)
     for x in inp.x_chunks:
         orc.append(x)
