@@ -599,7 +599,8 @@ def run_workload(args):
                 fms = _time(lambda: V.latent_attention_fused(cfg, qn, qr, wuk, wuv, cache, f0, out=o_f), 20, stream)
                 row.update({"fused_ms": fms, "fused_attention_tflops": attention_flops(cfg, B) / (fms * 1e-3) / 1e12})
                 ms = fms
-            if args.workload == "batch8":
+            if args.workload == "batch8" or d_c == dcs[-1]:
+                # dense MHA (per-head K, V: independent of d_c) on the same shapes and batch
                 w_kv = synthetic.draw_dense_weights(cfg, 77).to(dev)
                 dcache = V.DenseCache(cfg, B, device=dev)
                 for x in inp.x_chunks:
@@ -617,6 +618,14 @@ def run_workload(args):
             rows.append(row)
             del cache
             torch.cuda.empty_cache()
+        if args.workload == "dc_sweep":
+            # every rank against the one dense measurement (taken with the last row)
+            dms = rows[-1]["dense_mha_ms"]
+            for row in rows:
+                lat = row.get("fused_ms", row["latent_attention_ms"])
+                row.update({"dense_mha_ms": dms, "attention_time_ratio_latent_over_dense": lat / dms,
+                            "attention_alone_ratio_latent_over_dense": row["latent_attention_ms"] / dms,
+                            "ratio_uses": "fused call (absorb + attention + value-up) vs dense MHA"})
         out["rows"] = rows
     elif args.workload == "fewstep":
         out.update(_fewstep_workload(V, synthetic, dev, stream, clocks))
