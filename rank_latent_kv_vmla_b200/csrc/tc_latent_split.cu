@@ -18,9 +18,9 @@
 //               into one of two TMEM S buffers; for each key half w: O_w += P_{j-1,w} V_{j-1,w}, V = the
 //               c boxes read MN-major; (fused) o = (O / l) W^V_up,h^T at the end;
 //   warps 0-7   (fused) RoPE3D(q^rope) and q~ as bf16 into the Q buffer; softmax of one key half (one
-//               thread per query row = TMEM lane): masked running max with a lazy rescale of O_w, exp2 (a
-//               quarter by the FMA-pipe polynomial), row sum, P to TMEM in two parts of 32 keys; finally
-//               (max, sum) swapped through shared memory, and each warpgroup forms half of the columns of
+//               thread per query row = TMEM lane): masked running max with a lazy rescale of O_w, exp2
+//               (a quarter, three eighths in the fused call, by the FMA-pipe polynomial), row sum, P to
+//               TMEM in two parts of 32 keys; finally (max, sum) swapped through shared memory, and each warpgroup forms half of the columns of
 //               (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / l: stored (three-call) or written as bf16 into the Q
 //               buffer for the value up-projection, whose output each warpgroup then stores half of.
 // Three-call rows are (token, head) rows of q_abs (every head shares the KV tiles); fused tiles are 128
@@ -51,7 +51,6 @@ constexpr int kAuxBytes = 512;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 2 * kBN;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
-constexpr int kPolyPairs = 2;                 // of 8 score pairs per 16 keys: FMA-pipe 2^x
 constexpr int kPParts = 2;                    // each key half releases its P in two parts
 constexpr int kStepsPerPart = kHalf / 16 / kPParts;
 
@@ -102,6 +101,10 @@ latent_split_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_cons
   using PL = SplitPlan<KB, FUSED>;
   constexpr int NST = PL::kStages;
   constexpr int DV = PL::kDV;
+  // of the 8 score pairs per 16 keys, how many take the FMA-pipe 2^x (measured on B200 at batch 16,
+  // d_c = 64 / 128: three pairs 4-5 % faster than two for the fused call, within 1 % either way for
+  // the three-call attention; four slower for both)
+  constexpr int kPolyPairs = FUSED ? 3 : 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
