@@ -50,9 +50,10 @@ constexpr int kBlockM = 128;           // query rows per CTA
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Of the 8 score pairs in each 16-key chunk, this many take 2^x from the FMA-pipe polynomial
-// (exp2_poly2) and the rest from MUFU.EX2, which one warp per SM sub-partition would otherwise saturate.
+// (exp2_poly2) and the rest from MUFU.EX2, which one warp per SM sub-partition would otherwise saturate
+// (three: 1-1.8 % faster than two at d_c = 192 in interleaved runs on B200, four no better).
 #ifndef VMLA_EXP2_POLY_PAIRS
-#define VMLA_EXP2_POLY_PAIRS 2
+#define VMLA_EXP2_POLY_PAIRS 3
 #endif
 constexpr int kPolyPairs = VMLA_EXP2_POLY_PAIRS;
 // P of a tile is released to the P V MMAs in this many parts (consecutive key ranges), so that the
