@@ -12,7 +12,7 @@
 //               O += P_{j-1} V_{j-1} with P read from TMEM (it overwrites S_{j-1} as bf16);
 //   warps 0-3   one thread per query row (= TMEM lane): first the Q row into TMEM (when Q is kept
 //               in TMEM), then per tile the softmax: masked running max with a lazy rescale of O (only
-//               when the max grows by more than 2^8), exp2 (a quarter of them by an FMA-pipe
+//               when the max grows by more than 2^8), exp2 (3/8 of them by an FMA-pipe
 //               polynomial), row sum, P to TMEM in four parts of 32 keys, each released to the P V
 //               MMAs by its own barrier; finally O / l to global memory and the log-sum-exp.  The softmax is
 //               latency-bound with one warp per SM sub-partition, so it uses 3-input max and packed
