@@ -98,3 +98,40 @@ def test_rows_calls_reject_bad_ranges(V):
         V.latent_attention_fused_rows(cfg, qn, qr, wuk, wuv, cache, 0, cfg.chunk_tokens - 32)
     torch.cuda.synchronize()
     assert V.device_status() == 0
+
+
+def test_paired_compress_into_two_replicas_equals_single_call(V):
+    """At Wan shapes with B = 4 the compress runs on CTA pairs (M = 256 MMAs).  With two destination
+    rings (as when one replica is another GPU's; here both in this GPU's memory) every store of the
+    epilogue goes to both: the whole-chunk call into two replicas equals the one-destination call bit
+    for bit.  The same chunk split unevenly into two calls, as two ranks would issue them (narrower
+    tiles, no pairs), agrees within bf16 rounding."""
+    from rank_latent_kv_vmla_b200.config import WAN
+    cfg, B = WAN, 4
+    inp = synthetic.draw_layer(cfg, batch=B, seed=4242, n_chunks=2)
+    w = _to(inp.w_dkv_kr)
+    single = V.LatentCache(cfg, B, device=DEV, fill=float("nan"))
+    whole = [V.LatentCache(cfg, B, device=DEV, fill=float("nan")) for _ in range(2)]
+    split = [V.LatentCache(cfg, B, device=DEV, fill=float("nan")) for _ in range(2)]
+    cut = 2600                                 # not a multiple of 128 or 256
+    for x in inp.x_chunks:
+        f0 = single.frames_written
+        xd = _to(x)
+        V.compress_append(cfg, xd, w, single)
+        V.compress_append_rows(cfg, xd, w, f0, 0, [r.struct for r in whole], B)
+        for b0, cnt in ((0, cut), (cut, cfg.chunk_tokens - cut)):
+            V.compress_append_rows(cfg, xd[:, b0:b0 + cnt].contiguous(), w, f0, b0, [r.struct for r in split], B)
+        for r in whole + split:
+            r.struct.frames_written = single.frames_written
+    torch.cuda.synchronize()
+    assert V.device_status() == 0
+    rows = 2 * cfg.chunk_tokens
+    bits = lambda t: t.view(torch.int16)      # the unwritten rows are NaN: compare bit patterns
+    for r in whole:
+        assert torch.equal(bits(r.c), bits(single.c)) and torch.equal(bits(r.k_r), bits(single.k_r))
+    assert torch.equal(bits(split[0].c), bits(split[1].c)) and torch.equal(bits(split[0].k_r), bits(split[1].k_r))
+    for b in (0, B - 1):
+        for got, ref in ((split[0].c[b, :rows], single.c[b, :rows]), (split[0].k_r[b, :rows], single.k_r[b, :rows])):
+            rel_l2, _ = errors(f64(got), f64(ref))
+            assert rel_l2 <= 1e-3
+    assert torch.isnan(split[0].c[:, rows:].float()).all()
