@@ -117,9 +117,10 @@ def test_large_frame_index_fp32(V):
          check_from=cfg.window_frames)
 
 
-def test_whole_window_block_causal(V):
+@pytest.mark.parametrize("d_c", [192, 64])
+def test_whole_window_block_causal(V, d_c):
     """All W/F chunks of a window as one query set: chunk k sees chunks 0..k only."""
-    cfg = MID.replace(window_frames=6)
+    cfg = MID.replace(window_frames=6, d_c=d_c)
     n = cfg.window_frames // cfg.chunk_frames
     inp = synthetic.draw_layer(cfg, batch=2, seed=67, n_chunks=n, n_query_chunks=n)
     orc = OracleLayer(cfg, inp, 2)

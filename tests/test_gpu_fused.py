@@ -89,8 +89,9 @@ def test_mid_fused_narrow_heads(V):
     _stream_fused(V, MID.replace(d_nope=64, d_v=64), batch=1, n_steps=3, seed=3200)
 
 
-def test_mid_fused_block_causal_multichunk(V):
-    cfg = MID.replace(window_frames=8)
+@pytest.mark.parametrize("d_c", [192, 64, 128])
+def test_mid_fused_block_causal_multichunk(V, d_c):
+    cfg = MID.replace(window_frames=8, d_c=d_c)
     n = 3
     inp = synthetic.draw_layer(cfg, batch=1, seed=3300, n_chunks=n, n_query_chunks=n)
     orc = OracleLayer(cfg, inp, 1)
@@ -106,10 +107,11 @@ def test_mid_fused_block_causal_multichunk(V):
     assert_close(f64(lse[0]), ref["lse"], cfg, "lse")
 
 
-def test_mid_fused_peaked_softmax(V):
+@pytest.mark.parametrize("d_c", [192, 64])
+def test_mid_fused_peaked_softmax(V, d_c):
     """Logits x8: the running max moves and O is rescaled; compared with the three-call path on the
     same cache (the oracle comparison of this case is made call by call in test_gpu_parity)."""
-    cfg = MID
+    cfg = MID.replace(d_c=d_c)
     inp = synthetic.draw_layer(cfg, batch=1, seed=3400, n_chunks=3, q_gain=8.0)
     cache = V.LatentCache(cfg, 1, device=DEV)
     for x in inp.x_chunks:
@@ -156,11 +158,12 @@ def test_wan_fused_full_size_sampled(V):
         assert rel_l2 <= paths_rel_tol(cfg), (b, max_rel, rel_l2)
 
 
-def test_fused_bounded_wait_reports_timeout_and_context_survives(V):
+@pytest.mark.parametrize("d_c", [192, 64, 128])
+def test_fused_bounded_wait_reports_timeout_and_context_survives(V, d_c):
     """A KV tile the fused kernel never loads: the bounded wait runs out, every role winds down (the
     up-projection weights are not loaded, no output is written), vmla_device_status reports the code,
-    and the next fused call on the same context is correct."""
-    cfg = MID
+    and the next fused call on the same context is correct.  d_c = 64 / 128 run the key-split kernel."""
+    cfg = MID.replace(d_c=d_c)
     inp = synthetic.draw_layer(cfg, batch=1, seed=3600, n_chunks=3)
     cache = V.LatentCache(cfg, 1, device=DEV)
     for x in inp.x_chunks:

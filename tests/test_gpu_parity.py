@@ -139,9 +139,10 @@ def test_mid_bf16_attention_isolated_latent_sizes(V, d_c):
     _isolated_attention_and_value_up(V, MID.replace(d_c=d_c), seed=98 + d_c, batch=1)
 
 
-def test_mid_bf16_block_causal_multichunk(V):
+@pytest.mark.parametrize("d_c", [192, 64, 128])
+def test_mid_bf16_block_causal_multichunk(V, d_c):
     """One call over 3 query chunks (bidirectional inside a chunk, causal across chunks)."""
-    cfg = MID.replace(window_frames=8)
+    cfg = MID.replace(window_frames=8, d_c=d_c)
     n = 3
     inp = synthetic.draw_layer(cfg, batch=1, seed=7, n_chunks=n, n_query_chunks=n)
     orc = OracleLayer(cfg, inp, 1)
