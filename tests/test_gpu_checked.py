@@ -1,7 +1,8 @@
 """The bounds-checked build (libvmla_checked.so, VMLA_CHECKED=1), run in a child process: every
 computed global store of the tensor-core kernels is tested against its buffer's extent.  Every call of
-the path, the dense layer, the rewrite, the row-range (sharded) calls and the executor must run with
-no store outside its buffer; with the recorded extents shortened by one 32-column chunk
+the path, the dense layer, the rewrite, the row-range (sharded) calls, the executor, the key-split
+kernels (d_c 64 / 128) and the paired-CTA compress (Wan shapes, B = 4) must run with no store outside
+its buffer; with the recorded extents shortened by one 32-column chunk
 (vmla_debug_shrink_extents) the stores at the buffers' ends must be reported instead (and skipped)."""
 import os
 import subprocess
@@ -61,6 +62,26 @@ with V.Executor(cfg, B) as ex:
         ex.submit(lc, w, wuk, wuv, *hosts, ho)
     ex.wait()
 assert status("executor") == 0
+# the key-split attention kernels (d_c 64 / 128) and the paired-CTA compress (Wan shapes at B = 4)
+from rank_latent_kv_vmla_b200.config import WAN
+for d_c in (64, 128):
+    c2 = MID.replace(d_c=d_c)
+    w2, wuk2, wuv2 = (t.to(dev) for t in synthetic.draw_weights(c2, 5))
+    l2 = V.LatentCache(c2, B, device=dev)
+    for k in range(4):
+        x, qn, qr = (t.to(dev) for t in synthetic.draw_chunk(c2, B, 40 + k))
+        f0 = l2.frames_written
+        V.compress_append(c2, x, w2, l2)
+        V.latent_attention(c2, V.absorb_q(c2, qn, qr, wuk2, f0), l2, f0, want_lse=True)
+        V.latent_attention_fused(c2, qn, qr, wuk2, wuv2, l2, f0, want_lse=True)
+    assert status(f"key-split d_c {d_c}") == 0
+cw, bw = WAN, 4
+ww = synthetic.draw_weights(cw, 6)[0].to(dev)
+lw = V.LatentCache(cw, bw, device=dev)
+xw = [synthetic.draw_chunk(cw, bw, 50 + k)[0].to(dev) for k in range(2)]
+for k in range(7):                       # 7 chunks of 3 frames fill the 21-frame ring to its last row
+    V.compress_append(cw, xw[k % 2], ww, lw)
+assert status("paired compress") == 0
 # extents one 32-column chunk short: the stores at the ends are reported, codes 90 + site
 V.LIB.vmla_debug_shrink_extents(64)
 x, qn, qr = (t.to(dev) for t in synthetic.draw_chunk(cfg, B, 30))
@@ -70,10 +91,13 @@ V.compress_append(cfg, x, w, lc)
 code_c = status("shrunk compress")
 V.latent_attention_fused(cfg, qn, qr, wuk, wuv, lc, f0)
 code_a = status("shrunk fused attention")
+lw.struct.frames_written = 18            # the paired compress rewrites the ring's last chunk
+V.compress_append(cw, xw[0], ww, lw)
+code_p = status("shrunk paired compress")
 V.LIB.vmla_debug_shrink_extents(0)
 V.latent_attention_fused(cfg, qn, qr, wuk, wuv, lc, f0)
 assert status("restored") == 0
-print("CODES", code_c, code_a)
+print("CODES", code_c, code_a, code_p)
 """
 
 
@@ -88,6 +112,7 @@ def test_checked_build_finds_no_store_outside_its_buffer():
                        text=True, timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr
     codes = [l for l in r.stdout.splitlines() if l.startswith("CODES")][0].split()[1:]
-    code_c, code_a = int(codes[0]), int(codes[1])
+    code_c, code_a, code_p = int(codes[0]), int(codes[1]), int(codes[2])
     assert code_c in (91, 92), r.stdout          # c or k_r plane of the newest chunk's last slot
     assert code_a == 99, r.stdout                # the fused kernel's last output chunk
+    assert code_p in (91, 92), r.stdout          # the paired compress, same sites
