@@ -979,7 +979,9 @@ def main():
                  "clocks": nvml.window("sustained")}
     assert V.device_status() == 0
 
-    # ---- dense per-head MHA comparison on the same shapes (not part of `value`) ----
+    # ---- dense per-head MHA comparison on the same shapes (not part of `value`): dense and latent steps
+    # interleaved (latent, dense, dense, latent, ...) so that both see the same clock and power state;
+    # each arm's median over its steps ----
     comparison = None
     if not args.no_dense:
         w_kv = synthetic.draw_dense_weights(cfg, seed + 3).to(dev)
@@ -989,7 +991,6 @@ def main():
         dq = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_h), dtype=torch.bfloat16, device=dev)
         do = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
         dsteps = max(10, args.steps // 4)
-        devs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(dsteps)]
 
         def dstep(i, ev):
             f0 = dcache.frames_written
@@ -1002,21 +1003,35 @@ def main():
             ev[3].record(stream)
 
         # the dense cache (201 MB per sequence) alone exceeds L2
+        warm = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         for i in range(3):
-            dstep(i, devs[0])
+            dstep(i, warm)
             between_steps()
-        for i in range(dsteps):
-            dstep(i, devs[i])
+        lat0 = args.warmup + args.steps + 2 * ab_steps + sus_steps
+        d_ev, l_ev = [], []
+        for i in range(2 * dsteps):
+            if (i % 4) in (0, 3):
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+                step(lat0 + i, ev)
+                l_ev.append(ev)
+            else:
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                dstep(i, ev)
+                d_ev.append(ev)
             between_steps()
         torch.cuda.synchronize()
-        d_step_ms = statistics.mean(devs[i][0].elapsed_time(devs[i][3]) for i in range(dsteps))
-        d_mha_ms = statistics.mean(devs[i][2].elapsed_time(devs[i][3]) for i in range(dsteps))
+        d_step_ms = statistics.median(ev[0].elapsed_time(ev[3]) for ev in d_ev)
+        d_mha_ms = statistics.median(ev[2].elapsed_time(ev[3]) for ev in d_ev)
+        l_step_ms = statistics.median(ev[0].elapsed_time(ev[n_ev - 1]) for ev in l_ev)
+        k3i = names.index(k3)
+        l_k3_ms = statistics.median(ev[k3i].elapsed_time(ev[k3i + 1]) for ev in l_ev)
         comparison = {"dense_step_ms": d_step_ms, "dense_mha_ms": d_mha_ms,
                       "dense_mha_tflops": dense_attention_flops(cfg, B) / (d_mha_ms * 1e-3) / 1e12,
-                      "latent_step_ms": statistics.mean(step_ms), "latent_attention_ms": k3_ms,
+                      "latent_step_ms": l_step_ms, "latent_attention_ms": l_k3_ms,
                       "latent_attention_includes_projections": fused,
-                      "step_speedup_vs_dense": d_step_ms / statistics.mean(step_ms),
-                      "attention_speedup_vs_dense": d_mha_ms / k3_ms,
+                      "step_speedup_vs_dense": d_step_ms / l_step_ms,
+                      "attention_speedup_vs_dense": d_mha_ms / l_k3_ms,
+                      "how": f"{dsteps} dense and {dsteps} latent steps interleaved, medians",
                       "cache_bytes_latent": V.latent_cache_bytes(cfg, B),
                       "cache_bytes_dense": V.dense_cache_bytes(cfg, B),
                       "cache_bytes_ratio": V.latent_cache_bytes(cfg, B) / V.dense_cache_bytes(cfg, B)}
