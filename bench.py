@@ -459,6 +459,21 @@ def _time(fn, reps, stream):
     return statistics.mean(a.elapsed_time(b) for a, b in evs)
 
 
+def _time_pair(fa, fb, reps, stream):
+    """Median device times (ms) of fa() and fb(), reps calls each, interleaved a, b, b, a, ... so that
+    both see the same clock and power state."""
+    res = ([], [])
+    for i in range(2 * reps):
+        k = 0 if (i % 4) in (0, 3) else 1
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        (fa, fb)[k]()
+        b.record(stream)
+        res[k].append((a, b))
+    torch.cuda.synchronize()
+    return tuple(statistics.median(a.elapsed_time(b) for a, b in r) for r in res)
+
+
 def _fewstep_workload(V, synthetic, dev, stream, clocks, batch=1, n_chunks=14, n_denoise=4):
     """One Wan layer streaming n_chunks chunks, each denoised over n_denoise steps: the first step
     appends the chunk, the others rewrite it in place; every step attends with its own queries
@@ -472,40 +487,48 @@ def _fewstep_workload(V, synthetic, dev, stream, clocks, batch=1, n_chunks=14, n
     dq = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_h), dtype=torch.bfloat16, device=dev)
     res = {}
     clocks.start()
+    # the two layers step in lockstep, alternating which goes first, so that both see the same clock
+    caches = {"latent": V.LatentCache(cfg, B, device=dev), "dense": V.DenseCache(cfg, B, device=dev)}
+    f0 = {"latent": 0, "dense": 0}
+    evs = {"latent": [], "dense": []}
+
+    def one(path, k, s):
+        x, qn, qr = sets[s]
+        cache = caches[path]
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        if s == 0:
+            f0[path] = cache.frames_written
+        if path == "latent":
+            if s == 0:
+                V.compress_append(cfg, x, wd, cache)
+            else:
+                V.compress_rewrite(cfg, x, wd, cache)
+            V.latent_attention_fused(cfg, qn, qr, wuk, wuv, cache, f0[path], out=o)
+        else:
+            if s == 0:
+                V.dense_append(cfg, x, w_kv, cache)
+            else:
+                V.dense_rewrite(cfg, x, w_kv, cache)
+            V.rope_q(cfg, qn, qr, f0[path], out=dq)
+            V.dense_mha(cfg, dq, cache, f0[path], out=o)
+        b.record(stream)
+        evs[path].append((k, a, b))
+
+    for k in range(n_chunks):
+        for s in range(n_denoise):
+            for path in (("latent", "dense") if (k * n_denoise + s) % 2 == 0 else ("dense", "latent")):
+                one(path, k, s)
+    torch.cuda.synchronize()
     for path in ("latent", "dense"):
-        cache = V.LatentCache(cfg, B, device=dev) if path == "latent" else V.DenseCache(cfg, B, device=dev)
-        evs = []
-        for k in range(n_chunks):
-            for s in range(n_denoise):
-                x, qn, qr = sets[s]
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                if path == "latent":
-                    if s == 0:
-                        f0 = cache.frames_written
-                        V.compress_append(cfg, x, wd, cache)
-                    else:
-                        V.compress_rewrite(cfg, x, wd, cache)
-                    V.latent_attention_fused(cfg, qn, qr, wuk, wuv, cache, f0, out=o)
-                else:
-                    if s == 0:
-                        f0 = cache.frames_written
-                        V.dense_append(cfg, x, w_kv, cache)
-                    else:
-                        V.dense_rewrite(cfg, x, w_kv, cache)
-                    V.rope_q(cfg, qn, qr, f0, out=dq)
-                    V.dense_mha(cfg, dq, cache, f0, out=o)
-                b.record(stream)
-                evs.append((k, a, b))
-        torch.cuda.synchronize()
         # steady state: chunks whose window is full (frame f0 + F >= W)
-        full = [a.elapsed_time(b) for k, a, b in evs if (k + 1) * cfg.chunk_frames >= cfg.window_frames]
+        full = [a.elapsed_time(b) for k, a, b in evs[path] if (k + 1) * cfg.chunk_frames >= cfg.window_frames]
         ms = statistics.mean(full)
         fl = attention_flops(cfg, B) if path == "latent" else dense_attention_flops(cfg, B)
         res[path] = {"ms_per_denoising_step": ms, "attention_tflops_per_step_time": fl / (ms * 1e-3) / 1e12,
-                     "steps_timed": len(full), "total_ms_all_steps": sum(a.elapsed_time(b) for _, a, b in evs)}
-        del cache
-        torch.cuda.empty_cache()
+                     "steps_timed": len(full), "total_ms_all_steps": sum(a.elapsed_time(b) for _, a, b in evs[path])}
+    del caches
+    torch.cuda.empty_cache()
     res["step_time_ratio_latent_over_dense"] = res["latent"]["ms_per_denoising_step"] / res["dense"]["ms_per_denoising_step"]
     return {"batch": B, "chunks": n_chunks, "denoising_steps_per_chunk": n_denoise, **res}
 
@@ -519,7 +542,7 @@ def _capacity_workload(V, synthetic, dev, clocks, budget=60 * 10**9, n_layers=30
     for name, cfg, dense in (("latent_dc64", WAN.replace(d_c=64), False),
                              ("latent_dc128", WAN.replace(d_c=128), False),
                              ("latent_dc192", WAN, False), ("dense", WAN, True)):
-        # the latent step runs fused where the fused kernel supports the shape (d_c >= 128 here)
+        # the latent step runs fused where the fused kernel supports the shape
         fused = (not dense) and V.fused_supported(cfg)
         plan = V.plan_capacity(cfg, n_layers, budget, dense=dense, fused=fused)
         row = {"path": name + ("_fused" if fused else ""), **plan}
@@ -571,6 +594,20 @@ def run_workload(args):
         dcs = [192] if args.workload == "batch8" else [64, 128, 192]
         rows = []
         clocks.start()
+        # the dense MHA layer (per-head K, V: independent of d_c) on the same shapes and batch, timed
+        # interleaved with each latent call
+        inp_d = synthetic.draw_layer(WAN, batch=B, seed=1234 + 2, n_chunks=7)
+        w_kv = synthetic.draw_dense_weights(WAN, 77).to(dev)
+        dcache = V.DenseCache(WAN, B, device=dev)
+        for x in inp_d.x_chunks:
+            fd = dcache.frames_written
+            V.dense_append(WAN, x.to(dev), w_kv, dcache)
+        q_d = V.rope_q(WAN, inp_d.q_nope.to(dev), inp_d.q_rope.to(dev), fd)
+        o_d = torch.empty((B, WAN.chunk_tokens, WAN.n_heads, WAN.d_v), dtype=torch.bfloat16, device=dev)
+        dense_call = lambda: V.dense_mha(WAN, q_d, dcache, fd, out=o_d)
+        for _ in range(3):
+            dense_call()
+        del inp_d
         for d_c in dcs:
             cfg = WAN.replace(d_c=d_c)
             inp = synthetic.draw_layer(cfg, batch=B, seed=1234 + 2, n_chunks=7)
@@ -582,50 +619,36 @@ def run_workload(args):
             qn, qr, wuk = inp.q_nope.to(dev), inp.q_rope.to(dev), inp.w_uk.to(dev)
             q_abs = V.absorb_q(cfg, qn, qr, wuk, f0)
             o_lat = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_c), dtype=torch.bfloat16, device=dev)
+            lat_call = lambda: V.latent_attention(cfg, q_abs, cache, f0, out=o_lat)
             for _ in range(3):
-                V.latent_attention(cfg, q_abs, cache, f0, out=o_lat)
-            ms = _time(lambda: V.latent_attention(cfg, q_abs, cache, f0, out=o_lat), 20, stream)
+                lat_call()
+            ms, dms_a = _time_pair(lat_call, dense_call, 10, stream)
             row = {"d_c": d_c, "batch": B, "latent_attention_ms": ms,
                    "latent_tflops": attention_flops(cfg, B) / (ms * 1e-3) / 1e12,
                    "query_tokens_per_s": B * cfg.chunk_tokens / (ms * 1e-3),
                    "cache_bytes_per_layer": V.latent_cache_bytes(cfg, B),
-                   "cache_fraction_of_dense": V.latent_cache_bytes(cfg, B) / V.dense_cache_bytes(cfg, B)}
+                   "cache_fraction_of_dense": V.latent_cache_bytes(cfg, B) / V.dense_cache_bytes(cfg, B),
+                   "attention_alone_ratio_latent_over_dense": ms / dms_a}
+            dms = dms_a
             if V.fused_supported(cfg):
                 # the fused call: absorb + attention + value-up in one launch (what the layer step runs)
                 wuv = inp.w_uv.to(dev)
                 o_f = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
+                fused_call = lambda: V.latent_attention_fused(cfg, qn, qr, wuk, wuv, cache, f0, out=o_f)
                 for _ in range(3):
-                    V.latent_attention_fused(cfg, qn, qr, wuk, wuv, cache, f0, out=o_f)
-                fms = _time(lambda: V.latent_attention_fused(cfg, qn, qr, wuk, wuv, cache, f0, out=o_f), 20, stream)
+                    fused_call()
+                fms, dms = _time_pair(fused_call, dense_call, 10, stream)
                 row.update({"fused_ms": fms, "fused_attention_tflops": attention_flops(cfg, B) / (fms * 1e-3) / 1e12})
                 ms = fms
-            if args.workload == "batch8" or d_c == dcs[-1]:
-                # dense MHA (per-head K, V: independent of d_c) on the same shapes and batch
-                w_kv = synthetic.draw_dense_weights(cfg, 77).to(dev)
-                dcache = V.DenseCache(cfg, B, device=dev)
-                for x in inp.x_chunks:
-                    V.dense_append(cfg, x.to(dev), w_kv, dcache)
-                q = V.rope_q(cfg, qn, qr, f0)
-                o_d = torch.empty((B, cfg.chunk_tokens, cfg.n_heads, cfg.d_v), dtype=torch.bfloat16, device=dev)
-                for _ in range(3):
-                    V.dense_mha(cfg, q, dcache, f0, out=o_d)
-                dms = _time(lambda: V.dense_mha(cfg, q, dcache, f0, out=o_d), 20, stream)
-                row.update({"dense_mha_ms": dms, "dense_tflops": dense_attention_flops(cfg, B) / (dms * 1e-3) / 1e12,
-                            "attention_time_ratio_latent_over_dense": ms / dms,
-                            "ratio_uses": "fused call (absorb + attention + value-up) vs dense MHA",
-                            "dense_cache_bytes_per_layer": V.dense_cache_bytes(cfg, B)})
-                del dcache
+            row.update({"dense_mha_ms": dms, "dense_tflops": dense_attention_flops(cfg, B) / (dms * 1e-3) / 1e12,
+                        "attention_time_ratio_latent_over_dense": ms / dms,
+                        "ratio_uses": "fused call (absorb + attention + value-up) vs dense MHA, interleaved",
+                        "dense_cache_bytes_per_layer": V.dense_cache_bytes(cfg, B)})
             rows.append(row)
             del cache
             torch.cuda.empty_cache()
-        if args.workload == "dc_sweep":
-            # every rank against the one dense measurement (taken with the last row)
-            dms = rows[-1]["dense_mha_ms"]
-            for row in rows:
-                lat = row.get("fused_ms", row["latent_attention_ms"])
-                row.update({"dense_mha_ms": dms, "attention_time_ratio_latent_over_dense": lat / dms,
-                            "attention_alone_ratio_latent_over_dense": row["latent_attention_ms"] / dms,
-                            "ratio_uses": "fused call (absorb + attention + value-up) vs dense MHA"})
+        del dcache
+        torch.cuda.empty_cache()
         out["rows"] = rows
     elif args.workload == "fewstep":
         out.update(_fewstep_workload(V, synthetic, dev, stream, clocks))
