@@ -622,14 +622,18 @@ def run_workload(args):
             lat_call = lambda: V.latent_attention(cfg, q_abs, cache, f0, out=o_lat)
             for _ in range(3):
                 lat_call()
-            ms, dms_a = _time_pair(lat_call, dense_call, 10, stream)
+            # throughput: the latent calls timed on their own; comparison: each interleaved with the
+            # dense call (the dense kernel draws less power, so alternating with it changes the clock)
+            ms = _time(lat_call, 20, stream)
+            ms_i, dms_a = _time_pair(lat_call, dense_call, 10, stream)
             row = {"d_c": d_c, "batch": B, "latent_attention_ms": ms,
                    "latent_tflops": attention_flops(cfg, B) / (ms * 1e-3) / 1e12,
                    "query_tokens_per_s": B * cfg.chunk_tokens / (ms * 1e-3),
                    "cache_bytes_per_layer": V.latent_cache_bytes(cfg, B),
                    "cache_fraction_of_dense": V.latent_cache_bytes(cfg, B) / V.dense_cache_bytes(cfg, B),
-                   "attention_alone_ratio_latent_over_dense": ms / dms_a}
-            dms = dms_a
+                   "interleaved": {"latent_attention_ms": ms_i, "dense_mha_ms": dms_a},
+                   "attention_alone_ratio_latent_over_dense": ms_i / dms_a}
+            ms, dms = ms_i, dms_a
             if V.fused_supported(cfg):
                 # the fused call: absorb + attention + value-up in one launch (what the layer step runs)
                 wuv = inp.w_uv.to(dev)
@@ -637,8 +641,11 @@ def run_workload(args):
                 fused_call = lambda: V.latent_attention_fused(cfg, qn, qr, wuk, wuv, cache, f0, out=o_f)
                 for _ in range(3):
                     fused_call()
+                fms_alone = _time(fused_call, 20, stream)
                 fms, dms = _time_pair(fused_call, dense_call, 10, stream)
-                row.update({"fused_ms": fms, "fused_attention_tflops": attention_flops(cfg, B) / (fms * 1e-3) / 1e12})
+                row.update({"fused_ms": fms_alone,
+                            "fused_attention_tflops": attention_flops(cfg, B) / (fms_alone * 1e-3) / 1e12})
+                row["interleaved"].update({"fused_ms": fms, "dense_mha_ms_with_fused": dms})
                 ms = fms
             row.update({"dense_mha_ms": dms, "dense_tflops": dense_attention_flops(cfg, B) / (dms * 1e-3) / 1e12,
                         "attention_time_ratio_latent_over_dense": ms / dms,
